@@ -1,0 +1,113 @@
+"""Planted mistakes in copies of the oracle must each fail at least one pin.
+
+The mistakes are planted here, on the CPU, in the oracle's arithmetic (never in
+the CUDA path).  If a plausible slip (dropped scale, shifted mask, transposed
+operand, wrong sign, dropped term) passed every check, the checks would not be
+pinning the oracle.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import oracle_checks as oc
+
+
+def _fwd_generic(q, k, v, scale, causal, *, mask_strict=False, use_scale=True, lse_no_max=False,
+                 transpose=False, axis=-1, v_shift=False):
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    s = (k @ np.swapaxes(q, -1, -2)) if transpose else (q @ np.swapaxes(k, -1, -2))
+    if use_scale:
+        s = s * scale
+    N, Nk = s.shape[-2], s.shape[-1]
+    if causal:
+        j, i = np.meshgrid(np.arange(Nk), np.arange(N))
+        bad = (j >= i) & (j != 0) if mask_strict else (j > i)
+        s = np.where(bad, -np.inf, s)
+    m = s.max(axis=axis, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=axis, keepdims=True)
+    p = e / l
+    vv = np.roll(v, 1, axis=-2) if v_shift else v
+    o = p @ vv
+    lse = (np.log(l) if lse_no_max else m + np.log(l))
+    lse = lse[..., 0] if axis == -1 else np.broadcast_to(lse, s.shape)[..., 0]
+    return o, lse
+
+
+MUTANTS_FWD = {
+    "dropped_scale": dict(use_scale=False),
+    "mask_excludes_diagonal": dict(mask_strict=True),
+    "lse_without_max": dict(lse_no_max=True),
+    "transposed_scores": dict(transpose=True),
+    "softmax_wrong_axis": dict(axis=-2),
+    "v_rows_shifted": dict(v_shift=True),
+}
+
+
+def test_unmutated_generic_passes():
+    f = lambda q, k, v, s, c: _fwd_generic(q, k, v, s, c)
+    for chk in oc.FWD_CHECKS:
+        assert chk(f), chk.__name__
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS_FWD))
+def test_forward_mutant_is_caught(name):
+    kw = MUTANTS_FWD[name]
+    f = lambda q, k, v, s, c: _fwd_generic(q, k, v, s, c, **kw)
+    failures = []
+    for chk in oc.FWD_CHECKS:
+        try:
+            ok = chk(f)
+        except Exception:
+            ok = False
+        if not ok:
+            failures.append(chk.__name__)
+    assert failures, f"mutant {name} passed every forward check"
+
+
+def _bwd_generic(q, k, v, do, scale, causal, *, dk_unscaled=False, ds_sign=1.0, drop_D=False,
+                 dv_transposed=False):
+    q, k, v, do = (np.asarray(x, dtype=np.float64) for x in (q, k, v, do))
+    s = (q @ np.swapaxes(k, -1, -2)) * scale
+    N = s.shape[-1]
+    if causal:
+        s = np.where(np.triu(np.ones((N, N), bool), 1), -np.inf, s)
+    e = np.exp(s - s.max(-1, keepdims=True))
+    p = e / e.sum(-1, keepdims=True)
+    pt = np.swapaxes(p, -1, -2)
+    dv = (p @ do) if dv_transposed else (pt @ do)
+    dp = do @ np.swapaxes(v, -1, -2)
+    D = 0.0 if drop_D else (p * dp).sum(-1, keepdims=True)
+    ds = ds_sign * p * (dp - D)
+    dq = scale * ds @ k
+    dk = (1.0 if dk_unscaled else scale) * np.swapaxes(ds, -1, -2) @ q
+    return dq, dk, dv
+
+
+MUTANTS_BWD = {
+    "dk_missing_scale": dict(dk_unscaled=True),
+    "ds_sign_flipped": dict(ds_sign=-1.0),
+    "D_term_dropped": dict(drop_D=True),
+    "dv_uses_P_not_PT": dict(dv_transposed=True),
+}
+
+
+def test_unmutated_generic_bwd_passes():
+    f = lambda *a: _bwd_generic(*a)
+    for chk in oc.BWD_CHECKS:
+        assert chk(f), chk.__name__
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS_BWD))
+def test_backward_mutant_is_caught(name):
+    kw = MUTANTS_BWD[name]
+    f = lambda *a: _bwd_generic(*a, **kw)
+    failures = []
+    for chk in oc.BWD_CHECKS:
+        try:
+            ok = chk(f)
+        except Exception:
+            ok = False
+        if not ok:
+            failures.append(chk.__name__)
+    assert failures, f"mutant {name} passed every backward check"
