@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extras]
+
+Headline step: one bf16 causal forward of the workload B=4, H=16, N=4096, d=128
+(scale 1/sqrt(128), 1% of K rows x8), i.e. one fa_fwd launch over inputs already
+resident in HBM (Q, K, V = 201 MB > the 126 MB L2, so no flush is needed between
+steps).  Metric: attention TFLOP/s, counting 4*B*H*N^2*d halved for causal.
+
+Extra lines (same JSON object, key "extras"): forward+backward TFLOP/s for
+B=1 H=8 N=8192 d=64 causal and B=2 H=8 N=16384 d=256, and the FP8 forward for
+B=1 H=32 N=32768 d=128 causal (backward counted as 2.5x forward).
+
+With N GPUs (torchrun, one process per GPU) every rank runs its own copy of the
+workload (independent heads: no data-path collective); value = all ranks' FLOPs
+/ max-over-ranks time.  ``--impl reference`` times the fp64 CPU oracle on a
+bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+HEADLINE = "fwd_d128"
+METRIC = "attention TFLOP/s fwd and fwd+bwd on 1 B200; % of dense BF16/FP8 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes (read + write) per launch of the forward kernel at the headline workload,
+# from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` (profiles/
+# fa_fwd_d128_causal_B4H16N4096.md).  None until a capture of the current kernel exists.
+FWD_TRAFFIC_BYTES = None
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def time_steps(fn, steps, warmup, stream):
+    """Warm up, then time exactly `steps` calls with CUDA events on `stream`."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    per = []
+    start_all = torch.cuda.Event(enable_timing=True)
+    end_all = torch.cuda.Event(enable_timing=True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    start_all.record(stream)
+    for a, b in evs:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    end_all.record(stream)
+    torch.cuda.synchronize()
+    per = [a.elapsed_time(b) for a, b in evs]
+    return start_all.elapsed_time(end_all), per
+
+
+# ------------------------------------------------------------------ our implementation
+def run_ours(args):
+    import exact_attention_132_b200 as fa
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist  # noqa: F811
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    w = workloads.WORKLOADS[HEADLINE]
+
+    # inputs: seeded synthetic recipe, generated on the host, resident in HBM before timing
+    q, k, v = workloads.make_bf16_inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    step = lambda: fa.fa_fwd(qd, kd, vd, o, lse, scale=w.sm_scale, causal=True, stream=stream)
+
+    clocks = ClockSampler(local)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    total_ms, per = time_steps(step, args.steps, args.warmup, stream)
+    clk = clocks.stop()
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    flops = w.fwd_flops()
+    value = flops * args.steps * world / (total_ms * 1e-3) / 1e12
+    kernel_ms = statistics.mean(per)
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+
+    # end to end through the public API with host buffers: H2D of Q, K, V from pinned
+    # memory, the forward, D2H of O and LSE, every step
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        fa.fa_fwd(qd, kd, vd, o, lse, scale=w.sm_scale, causal=True, stream=stream)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_ms, _ = time_steps(e2e_step, e2e_steps, 2, stream)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    extras = {}
+    if not args.no_extras:
+        extras = run_extras(fa, dev, stream, max(3, min(args.steps, 10)), peak)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16; 1% of K rows x8)",
+        "config": {"workload": "bf16 causal forward B=4 H=16 N=4096 d=128 scale=1/sqrt(128)",
+                   "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True,
+                   "global_batch": w.B * world, "seq_len": w.N,
+                   "parallelism": f"replicas x{world} (independent heads, no collective)",
+                   "l2": "inputs 201 MB > 126 MB L2; no flush"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_src} bf16 dense matmul (burst)",
+                     "kernel": "fa_fwd_kernel<FwdCfg<128,128,2,false>>",
+                     "kernel_ms": round(kernel_ms, 4),
+                     "traffic": FWD_TRAFFIC_BYTES},
+        "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "ms_per_step": round(e2e_ms / e2e_steps, 4)},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+        "extras": extras,
+    }
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_extras(fa, dev, stream, steps, peak):
+    """fwd+bwd at the two backward workloads and the FP8 forward; device-side seeded inputs."""
+    out = {}
+    gen = torch.Generator(device=dev)
+    for name in ("fwdbwd_d64", "fwdbwd_d256"):
+        w = workloads.WORKLOADS[name]
+        gen.manual_seed(w.seed)
+        shp = (w.B, w.H, w.N, w.d)
+        q, k, v, do = ((torch.randn(shp, generator=gen, device=dev) * w.std).to(torch.bfloat16)
+                       for _ in range(4))
+        o = torch.empty_like(q)
+        lse = torch.empty(shp[:3], dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(max(1, fa.fa_bwd_workspace_size(*shp)), dtype=torch.uint8, device=dev)
+
+        def fb():
+            fa.fa_fwd(q, k, v, o, lse, scale=w.sm_scale, causal=w.causal, stream=stream)
+            fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale=w.sm_scale, causal=w.causal,
+                      stream=stream)
+
+        def fwd_only():
+            fa.fa_fwd(q, k, v, o, lse, scale=w.sm_scale, causal=w.causal, stream=stream)
+
+        tot, _ = time_steps(fb, steps, 2, stream)
+        ftot, _ = time_steps(fwd_only, steps, 2, stream)
+        fl = w.fwd_flops() + w.bwd_flops()
+        out[name] = {"workload": f"B={w.B} H={w.H} N={w.N} d={w.d} "
+                                 f"{'causal' if w.causal else 'non-causal'} fwd+bwd",
+                     "tflops_fwd_bwd": round(fl * steps / (tot * 1e-3) / 1e12, 2),
+                     "tflops_fwd": round(w.fwd_flops() * steps / (ftot * 1e-3) / 1e12, 2),
+                     "tflops_bwd": round(w.bwd_flops() * steps / ((tot - ftot) * 1e-3) / 1e12, 2)
+                     if tot > ftot else None,
+                     "ms_fwd_bwd": round(tot / steps, 3), "ms_fwd": round(ftot / steps, 3),
+                     "frac_of_bf16_peak": round(fl * steps / (tot * 1e-3) / 1e12 / peak, 4)}
+        del q, k, v, do, o, dq, dk, dv, ws
+    w = workloads.WORKLOADS["fp8_d128"]
+    gen.manual_seed(w.seed)
+    shp = (w.B, w.H, w.N, w.d)
+    nt = (w.N + 127) // 128
+    t8, sc = {}, {}
+    for n in "qkv":
+        x = torch.randn(shp, generator=gen, device=dev).view(w.B, w.H, nt, 128, w.d)
+        s = (x.abs().amax(dim=(3, 4)) / 448.0).clamp_min(1e-30)
+        t8[n] = (x / s[..., None, None]).clamp(-448, 448).to(torch.float8_e4m3fn).view(shp)
+        sc[n] = s.float().contiguous()
+        del x
+    o = torch.empty(shp, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(shp[:3], dtype=torch.float32, device=dev)
+    f8 = lambda: fa.fa_fwd_fp8(t8["q"], t8["k"], t8["v"], sc["q"], sc["k"], sc["v"], o, lse,
+                               scale=w.sm_scale, causal=True, stream=stream)
+    tot, _ = time_steps(f8, steps, 2, stream)
+    out["fp8_d128"] = {"workload": "FP8 e4m3 causal forward B=1 H=32 N=32768 d=128",
+                       "tflops_fwd": round(w.fwd_flops() * steps / (tot * 1e-3) / 1e12, 2),
+                       "ms_fwd": round(tot / steps, 3),
+                       "frac_of_fp8_nominal_2x_bf16_peak":
+                           round(w.fwd_flops() * steps / (tot * 1e-3) / 1e12 / (2 * peak), 4)}
+    return out
+
+
+# ------------------------------------------------------------------ CPU oracle
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, seconds):
+    """Time the fp64 oracle (as it stands) on whole heads of the workload until about
+    `seconds` of CPU work has been done; TFLOP/s in the workload's algorithmic count."""
+    import oracle
+    q, k, v = workloads.make_bf16_inputs(w)
+    per_head = w.fwd_flops() / (w.B * w.H)
+    heads, t0 = 0, time.perf_counter()
+    while True:
+        b, h = divmod(heads, w.H)
+        oracle.attention_fwd_heads(q, k, v, w.sm_scale, w.causal, [(b % w.B, h)])
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or heads >= w.B * w.H:
+            break
+    return {"value": round(per_head * heads / el / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(),
+            "kind": "oracle",
+            "sample": f"{heads} of {w.B * w.H} heads of the headline workload, all rows, fp64 NumPy, "
+                      f"{el:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = workloads.WORKLOADS[HEADLINE]
+    import oracle
+    q, k, v = workloads.make_bf16_inputs(w)
+    per_head = w.fwd_flops() / (w.B * w.H)
+    heads_per_step = max(1, args.ref_heads)
+
+    def one(step_idx):
+        for j in range(heads_per_step):
+            idx = (step_idx * heads_per_step + j) % (w.B * w.H)
+            b, h = divmod(idx, w.H)
+            oracle.attention_fwd_heads(q, k, v, w.sm_scale, True, [(b, h)])
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(args.warmup + i)
+    el = time.perf_counter() - t0
+    val = per_head * heads_per_step * args.steps / el / 1e12
+    sample = (f"{heads_per_step} head(s) of {w.B * w.H} per step (all 4096 rows), fp64 NumPy "
+              f"oracle on the host")
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) bf16; 1% of K rows x8)",
+            "config": {"workload": "bf16 causal forward B=4 H=16 N=4096 d=128 scale=1/sqrt(128)",
+                       "sample": sample},
+            "cpu_baseline": {"kind": "oracle", "cores": _cores(), "sample": sample,
+                             "value": round(val, 6), "unit": "TFLOP/s"},
+            "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-heads", type=int, default=1)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,195 @@
+"""Python binding of libfa.so: exact fused attention for B200 (sm_100a).
+
+Argument marshalling only: every function here checks shapes/dtypes, takes the
+device pointers and the current CUDA stream from torch, and calls the C entry
+point of the same name (declared in include/fa.h).  All arithmetic runs in the
+library's CUDA kernels; there is no Python or CPU fallback, and importing this
+package fails if the library has not been built
+(``python -m exact_attention_132_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "FAError", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_size", "fa_last_error_string",
+    "fa_get_device_status", "fa_debug_wait_timeout_selftest", "fa_version", "attention_forward",
+    "attention_forward_fp8", "attention_backward", "LIB_PATH", "lib",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT = range(5)
+STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
+                4: "FA_ERR_DEVICE_TIMEOUT"}
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m exact_attention_132_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    L.fa_bwd_workspace_size.restype = sz
+    L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
+    L.fa_last_error_string.argtypes = []
+    L.fa_last_error_string.restype = ctypes.c_char_p
+    L.fa_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    L.fa_debug_wait_timeout_selftest.argtypes = [i, vp]
+    L.fa_version.argtypes = []
+    for name in ("fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_get_device_status",
+                 "fa_debug_wait_timeout_selftest", "fa_version"):
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+def fa_last_error_string() -> str:
+    return lib.fa_last_error_string().decode()
+
+
+def _check(status: int) -> None:
+    if status != FA_OK:
+        raise FAError(status, fa_last_error_string())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _bhnd(t: torch.Tensor, name: str, dtype) -> tuple:
+    if t.dim() != 4:
+        raise ValueError(f"{name} must be [B, H, N, d], got shape {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    return tuple(t.shape)
+
+
+def fa_fwd(q, k, v, o, lse=None, scale: float | None = None, causal: bool = False, stream=None):
+    """O = softmax(scale Q K^T) V into ``o`` (bf16) and row logsumexp into ``lse`` (fp32)."""
+    B, H, N, d = _bhnd(q, "q", torch.bfloat16)
+    for t, n in ((k, "k"), (v, "v"), (o, "o")):
+        if _bhnd(t, n, torch.bfloat16) != (B, H, N, d):
+            raise ValueError(f"{n} shape differs from q")
+    if lse is not None and (tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32):
+        raise ValueError("lse must be fp32 [B, H, N]")
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, sc,
+                      1 if causal else 0, _stream(stream)))
+
+
+def fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse=None, scale: float | None = None,
+               causal: bool = False, stream=None):
+    """FP8 e4m3 forward with per-128-row-tile fp32 scales; bf16 output."""
+    B, H, N, d = _bhnd(q8, "q8", torch.float8_e4m3fn)
+    for t, n in ((k8, "k8"), (v8, "v8")):
+        if _bhnd(t, n, torch.float8_e4m3fn) != (B, H, N, d):
+            raise ValueError(f"{n} shape differs from q8")
+    if _bhnd(o, "o", torch.bfloat16) != (B, H, N, d):
+        raise ValueError("o shape differs from q8")
+    nt = (N + 127) // 128
+    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        if tuple(t.shape) != (B, H, nt) or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous fp32 [B, H, ceil(N/128)]")
+    if lse is not None and (tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32):
+        raise ValueError("lse must be fp32 [B, H, N]")
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale),
+                          _ptr(v_scale), _ptr(o), _ptr(lse), B, H, N, d, sc,
+                          1 if causal else 0, _stream(stream)))
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib.fa_bwd_workspace_size(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, scale: float | None = None,
+           causal: bool = False, stream=None):
+    """dQ, dK, dV (bf16) of L = sum(O * dO), recomputing P from the saved ``lse``."""
+    B, H, N, d = _bhnd(q, "q", torch.bfloat16)
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (dO, "dO"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if _bhnd(t, n, torch.bfloat16) != (B, H, N, d):
+            raise ValueError(f"{n} shape differs from q")
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be fp32 [B, H, N]")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk),
+                      _ptr(dv), _ptr(workspace), ws_bytes, B, H, N, d, sc, 1 if causal else 0,
+                      _stream(stream)))
+
+
+def fa_get_device_status(stream=None) -> int:
+    code = ctypes.c_int(0)
+    _check(lib.fa_get_device_status(_stream(stream), ctypes.byref(code)))
+    return code.value
+
+
+def fa_debug_wait_timeout_selftest(timeout_us: int, stream=None) -> None:
+    _check(lib.fa_debug_wait_timeout_selftest(int(timeout_us), _stream(stream)))
+
+
+def fa_version() -> int:
+    return int(lib.fa_version())
+
+
+# ------------------------------------------------------------------ allocating helpers
+def attention_forward(q, k, v, causal: bool = False, scale: float | None = None):
+    """Allocate O and LSE with torch and run fa_fwd; returns (o, lse)."""
+    B, H, N, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, o, lse, scale=scale, causal=causal)
+    return o, lse
+
+
+def attention_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal: bool = False,
+                          scale: float | None = None):
+    B, H, N, d = q8.shape
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, scale=scale, causal=causal)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, dO, lse, causal: bool = False, scale: float | None = None,
+                       workspace=None):
+    """Allocate dQ/dK/dV (and the workspace unless given) and run fa_bwd."""
+    B, H, N, d = q.shape
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        nbytes = fa_bwd_workspace_size(B, H, N, d)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, scale=scale, causal=causal)
+    return dq, dk, dv

@@ -1,0 +1,391 @@
+// fa_api.cu — the C ABI of libfa.so (declared in include/fa.h): argument
+// checks, TMA tensor-map construction, kernel selection by head dimension and
+// launches.  The library allocates no device memory on any call path.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+// Device status word written by kernels whose bounded waits expired.
+__device__ unsigned g_fa_status = 0;
+
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
+constexpr int kMaxDevices = 64;
+
+thread_local std::string t_last_error;
+
+fa_status fail(fa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+fa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------ per-device cache
+struct DeviceInfo {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  int sms = 0;
+  unsigned* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+fa_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_CUDA, "device index %d out of range", dev);
+  DeviceInfo& d = g_dev[dev];
+  std::call_once(d.once, [&] {
+    d.err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (d.err == cudaSuccess) {
+      int major = 0, minor = 0;
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+      if (major != 10 || minor != 0) d.err = cudaErrorNoKernelImageForDevice;
+    }
+    if (d.err == cudaSuccess)
+      d.err = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_fa_status);
+  });
+  if (d.err != cudaSuccess) return cuda_fail(d.err, "device setup (needs an sm_100 GPU)");
+  *out = &d;
+  return FA_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// [BH, N, d] row-major tensor seen as 3-D (d, N, BH); box = (inner, rows, 1) with
+// 128-byte swizzle.  Rows past N read as zero.
+fa_status make_map(CUtensorMap* m, const void* ptr, bool fp8, int d, int N, int BH, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  const int eb = fp8 ? 1 : 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * eb, static_cast<cuuint64_t>(N) * d * eb};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FA_OK;
+}
+
+// Set the dynamic shared-memory limit of a kernel once per device.
+template <class K>
+fa_status prepare_kernel(K kernel, int smem_bytes) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return FA_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_common(int B, int H, int N, float scale, bool* empty) {
+  if (B < 0 || H < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "negative size B=%d H=%d N=%d", B, H, N);
+  if (!std::isfinite(scale) || !(scale > 0.f))
+    return fail(FA_ERR_INVALID_ARG, "scale must be finite and > 0 (got %g)", static_cast<double>(scale));
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > (1ll << 30)) return fail(FA_ERR_INVALID_ARG, "B*H too large");
+  *empty = (bh == 0 || N == 0);
+  return FA_OK;
+}
+
+fa_status check_ptrs(const void* const* ptrs, const char* const* names, int n) {
+  for (int i = 0; i < n; ++i) {
+    if (ptrs[i] == nullptr) return fail(FA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned16(ptrs[i])) return fail(FA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  return FA_OK;
+}
+
+int causal_group_heads(int BH, long long kv_bytes_per_head) {
+  // heads whose K/V together fill about 32 MB of L2
+  long long g = (32ll << 20) / (kv_bytes_per_head > 0 ? kv_bytes_per_head : 1);
+  if (g < 1) g = 1;
+  if (g > BH) g = BH;
+  return static_cast<int>(g);
+}
+
+template <class C>
+fa_status launch_fwd(const void* q, const void* k, const void* v, FwdParams p, cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  if (fa_status s = device_info(&di)) return s;
+  CUtensorMap mq, mk, mv;
+  if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
+  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
+  auto kern = fa_fwd_kernel<C>;
+  if (fa_status s = prepare_kernel(kern, C::SMEM_ALLOC)) return s;
+  p.n_qt = (p.N + C::BM - 1) / C::BM;
+  p.n_kt = (p.N + C::BN - 1) / C::BN;
+  p.n_st = (p.N + 127) / 128;
+  p.total_items = p.BH * p.n_qt;
+  p.group_heads = causal_group_heads(p.BH, 2ll * p.N * C::D * C::ELEM);
+  p.status = di->status;
+  p.timeout_ns = kWaitTimeoutNs;
+  const int grid = p.total_items < di->sms ? p.total_items : di->sms;
+  kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
+  return FA_OK;
+}
+
+using FwdD64 = FwdCfg<64, 128, 3, false>;
+using FwdD128 = FwdCfg<128, 128, 2, false>;
+using FwdD256 = FwdCfg<256, 64, 2, false>;
+using FwdF8D128 = FwdCfg<128, 128, 3, true>;
+
+using DkdvD64 = DkdvCfg<64, 64, 128, 3>;
+using DkdvD128 = DkdvCfg<128, 128, 128, 2>;
+using DkdvD256 = DkdvCfg<256, 128, 64, 1>;
+using DqD64 = DqCfg<64, 128, 3>;
+using DqD128 = DqCfg<128, 128, 2>;
+using DqD256 = DqCfg<256, 64, 1>;
+
+template <class CK, class CQ>
+fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                     BwdParams p, cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  if (fa_status s = device_info(&di)) return s;
+  constexpr int D = CK::D;
+  p.status = di->status;
+  p.timeout_ns = kWaitTimeoutNs;
+  // 1. D_i = dO_i . O_i
+  {
+    const long long rows = static_cast<long long>(p.BH) * p.N;
+    constexpr int rpb = 256 / (D / 8);
+    long long blocks = (rows + rpb - 1) / rpb;
+    const long long cap = static_cast<long long>(di->sms) * 8;
+    if (blocks > cap) blocks = cap;
+    fa_bwd_rowdot<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO),
+        const_cast<float*>(p.drow), rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "row-dot kernel launch");
+  }
+  // 2. dK, dV
+  {
+    CUtensorMap mq, mk, mv, mdo;
+    if (fa_status s = make_map(&mq, q, false, D, p.N, p.BH, CK::BMQ)) return s;
+    if (fa_status s = make_map(&mdo, dO, false, D, p.N, p.BH, CK::BMQ)) return s;
+    if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH, CK::BN)) return s;
+    if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH, CK::BN)) return s;
+    auto kern = fa_bwd_dkdv<CK>;
+    if (fa_status s = prepare_kernel(kern, CK::SMEM_ALLOC)) return s;
+    BwdParams pk = p;
+    pk.n_qt = (p.N + CK::BMQ - 1) / CK::BMQ;
+    pk.n_kt = (p.N + CK::BN - 1) / CK::BN;
+    const long long grid = static_cast<long long>(p.BH) * pk.n_kt * CK::NSPLIT;
+    kern<<<static_cast<unsigned>(grid), CK::THREADS, CK::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, pk);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dK/dV kernel launch");
+  }
+  // 3. dQ
+  {
+    CUtensorMap mq, mk, mv, mdo;
+    if (fa_status s = make_map(&mq, q, false, D, p.N, p.BH, CQ::BM)) return s;
+    if (fa_status s = make_map(&mdo, dO, false, D, p.N, p.BH, CQ::BM)) return s;
+    if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH, CQ::BN)) return s;
+    if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH, CQ::BN)) return s;
+    auto kern = fa_bwd_dq<CQ>;
+    if (fa_status s = prepare_kernel(kern, CQ::SMEM_ALLOC)) return s;
+    BwdParams pq = p;
+    pq.n_qt = (p.N + CQ::BM - 1) / CQ::BM;
+    pq.n_kt = (p.N + CQ::BN - 1) / CQ::BN;
+    const long long grid = static_cast<long long>(p.BH) * pq.n_qt;
+    kern<<<static_cast<unsigned>(grid), CQ::THREADS, CQ::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, pq);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dQ kernel launch");
+  }
+  return FA_OK;
+}
+
+__global__ void wait_selftest_kernel(unsigned* status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtl wc{&abort_flag, status, timeout_ns};
+  // Nothing ever arrives on `bar`: the wait has to run out and report.
+  mbar_wait(smem_u32(&bar), 0, wc, kSiteSelfTest);
+  __syncthreads();
+}
+
+size_t workspace_bytes(int B, int H, int N) {
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                 int d, float scale, int causal, void* stream) {
+  bool empty = false;
+  if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
+  if (d != 64 && d != 128 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
+  if (empty) return FA_OK;
+  const void* ptrs[] = {q, k, v, o};
+  const char* names[] = {"q", "k", "v", "o"};
+  if (fa_status s = check_ptrs(ptrs, names, 4)) return s;
+  if (lse && !aligned16(lse)) return fail(FA_ERR_INVALID_ARG, "lse is not 16-byte aligned");
+  FwdParams p{};
+  p.BH = B * H;
+  p.N = N;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.o = o;
+  p.lse = lse;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_fwd<FwdD64>(q, k, v, p, st);
+    case 128: return launch_fwd<FwdD128>(q, k, v, p, st);
+    default: return launch_fwd<FwdD256>(q, k, v, p, st);
+  }
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,
+                     const float* k_scale, const float* v_scale, void* o, float* lse, int B, int H,
+                     int N, int d, float scale, int causal, void* stream) {
+  bool empty = false;
+  if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
+  if (d != 128) return fail(FA_ERR_UNSUPPORTED, "FP8 head dim %d not supported (128)", d);
+  if (empty) return FA_OK;
+  const void* ptrs[] = {q8, k8, v8, o};
+  const char* names[] = {"q8", "k8", "v8", "o"};
+  if (fa_status s = check_ptrs(ptrs, names, 4)) return s;
+  if (!q_scale || !k_scale || !v_scale) return fail(FA_ERR_INVALID_ARG, "FP8 scale pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale) |
+       reinterpret_cast<uintptr_t>(v_scale)) & 3u)
+    return fail(FA_ERR_INVALID_ARG, "FP8 scales must be 4-byte aligned");
+  if (lse && !aligned16(lse)) return fail(FA_ERR_INVALID_ARG, "lse is not 16-byte aligned");
+  FwdParams p{};
+  p.BH = B * H;
+  p.N = N;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.o = o;
+  p.lse = lse;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  return launch_fwd<FwdF8D128>(q8, k8, v8, p, static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  (void)d;
+  if (B <= 0 || H <= 0 || N <= 0) return 0;
+  return workspace_bytes(B, H, N);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes_, int B, int H, int N, int d, float scale, int causal,
+                 void* stream) {
+  bool empty = false;
+  if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
+  if (d != 64 && d != 128 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
+  if (empty) return FA_OK;
+  const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv, workspace};
+  const char* names[] = {"q", "k", "v", "o", "dO", "lse", "dq", "dk", "dv", "workspace"};
+  if (fa_status s = check_ptrs(ptrs, names, 10)) return s;
+  if (workspace_bytes_ < workspace_bytes(B, H, N))
+    return fail(FA_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes_,
+                workspace_bytes(B, H, N));
+  BwdParams p{};
+  p.BH = B * H;
+  p.N = N;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.lse = lse;
+  p.drow = static_cast<const float*>(workspace);
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_bwd<DkdvD64, DqD64>(q, k, v, o, dO, p, st);
+    case 128: return launch_bwd<DkdvD128, DqD128>(q, k, v, o, dO, p, st);
+    default: return launch_bwd<DkdvD256, DqD256>(q, k, v, o, dO, p, st);
+  }
+}
+
+const char* fa_last_error_string(void) { return t_last_error.c_str(); }
+
+fa_status fa_get_device_status(void* stream, int* code) {
+  if (!code) return fail(FA_ERR_INVALID_ARG, "code is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_fa_status, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  const unsigned zero = 0;
+  e = cudaMemcpyToSymbol(g_fa_status, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+  *code = static_cast<int>(v);
+  return FA_OK;
+}
+
+fa_status fa_debug_wait_timeout_selftest(int timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 2000000)
+    return fail(FA_ERR_INVALID_ARG, "timeout_us must be in [1, 2000000]");
+  DeviceInfo* di = nullptr;
+  if (fa_status s = device_info(&di)) return s;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      di->status, static_cast<unsigned long long>(timeout_us) * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return FA_OK;
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

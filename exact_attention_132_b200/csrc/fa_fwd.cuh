@@ -1,0 +1,454 @@
+// fa_fwd.cuh — fused attention forward for sm_100a (bf16 and FP8 e4m3 inputs).
+//
+// One persistent CTA per SM walks a static list of work items (b, h, 128-row
+// query tile).  For each item it streams the key/value tiles of that head:
+//
+//   S_j = Q K_j^T                      tcgen05.mma, fp32 accumulator in TMEM
+//   m'  = max(m, rowmax(S_j) * c)      c = scale * log2(e) (times the FP8 tile scales)
+//   P_j = 2^(S_j * c - m')             on the special-function unit, P written to TMEM
+//   l   = l * 2^(m - m') + rowsum(P_j)
+//   O   = O * 2^(m - m')               only for warps where some row max changed
+//   O  += P_j V_j                      tcgen05.mma with A = P from TMEM
+//
+// and finally O / l -> bf16 and lse = (m + log2 l) * ln 2.  This is the tiling +
+// online softmax + fusion of "FlashAttention — フラッシュアテンション" (wiki,
+// sections タイリングとブロック処理, オンラインSoftmax計算, CUDAカーネルの融合) and of
+// the issoh.co.jp page (sections QKVをブロック分割してSRAMへ載せるタイリングの手順 and
+// 最大値と正規化項を持ち回るオンラインsoftmaxの再スケール).  Rescaling only when the
+// max moves follows the same page's section on FA4 (FA4のB200で1613TFLOPs…:
+// "rescale only when needed").  Causal tiles wholly above the diagonal are
+// never visited (mypcrig.com post, section "FA2 の改善").
+//
+// Roles (warp specialisation, mypcrig.com post, section "FA3 の飛躍"):
+//   warp 0       TMA producer: Q tile per item, K/V tiles into a STAGES-deep ring
+//   warp 1       MMA issuer (one thread) + tensor-memory owner
+//   warps 2..5   softmax/correction/epilogue: thread t owns query row 32*(w%4)+lane,
+//                which is TMEM lane 32*(w%4)+lane (the lane quadrant a warp may use)
+//
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   [0, BN)      S buffer 0 (fp32); P of that step overwrites its first columns
+//   [BN, 2BN)    S buffer 1
+//   [2BN, 2BN+D) O accumulator (fp32)
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  int BH;             // B * H
+  int N;              // sequence length (queries = keys)
+  int n_qt;           // ceil(N / 128)
+  int n_kt;           // ceil(N / BN)
+  int n_st;           // ceil(N / 128): FP8 scale tiles per head
+  int causal;
+  int group_heads;    // causal ordering: heads that share one heaviest-first sweep
+  int total_items;    // BH * n_qt
+  float scale;        // multiplier of Q K^T
+  void* o;            // bf16 [BH, N, D]
+  float* lse;         // fp32 [BH, N] or null
+  const float* q_scale;   // FP8 only: [BH, n_st]
+  const float* k_scale;
+  const float* v_scale;
+  unsigned* status;
+  unsigned long long timeout_ns;
+};
+
+template <int D_, int BN_, int STAGES_, bool FP8_>
+struct FwdCfg {
+  static constexpr int D = D_;
+  static constexpr int BN = BN_;
+  static constexpr int STAGES = STAGES_;
+  static constexpr bool FP8 = FP8_;
+  static constexpr int BM = 128;
+  static constexpr int ELEM = FP8 ? 1 : 2;
+  static constexpr int ROW_BYTES = D * ELEM;        // bytes of one tile row
+  static constexpr int NBOX = ROW_BYTES / 128;      // 128-byte swizzle boxes per row
+  static constexpr int BOX_ELEMS = 128 / ELEM;
+  static constexpr int Q_BYTES = BM * ROW_BYTES;
+  static constexpr int KV_BYTES = BN * ROW_BYTES;
+  static constexpr int MMA_K = FP8 ? 32 : 16;       // K of one tcgen05.mma
+  static constexpr int KSTEP_BYTES = MMA_K * ELEM;  // always 32
+  static constexpr int SMEM_Q = 0;
+  static constexpr int SMEM_K = Q_BYTES;
+  static constexpr int SMEM_V = SMEM_K + STAGES * KV_BYTES;
+  static constexpr int SMEM_BAR = SMEM_V + STAGES * KV_BYTES;
+  // barriers
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_ODONE = 6,
+                       B_DRAIN = 7, B_KFULL = 8, B_VFULL = 8 + STAGES,
+                       B_KVEMPTY = 8 + 2 * STAGES, NBARS = 8 + 3 * STAGES;
+  static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;   // tmem slot, abort flag, reductions
+  static constexpr int SMEM_TOTAL = SMEM_MISC + 64;
+  static constexpr int SMEM_ALLOC = SMEM_TOTAL + 1024;     // slack to align the base to 1024
+  static constexpr int TM_S = 0;
+  static constexpr int TM_O = 2 * BN;
+  static constexpr int TM_COLS = 512;
+  static constexpr int P_COLS = BN * (FP8 ? 1 : 2) / 4;    // 32-bit columns holding P
+  static constexpr int THREADS = 192;
+  static_assert(2 * BN + D <= TM_COLS, "tensor memory budget");
+  static_assert(ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle rows");
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+  static_assert(BN % 32 == 0 && D % 32 == 0, "32-column TMEM chunks");
+};
+
+// Work item k of this CTA: rounds of gridDim.x items, alternate rounds walked in
+// reverse CTA order so the heaviest-first list evens out across CTAs.
+__device__ __forceinline__ int fwd_item_index(int k) {
+  const int pos = (k & 1) ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
+  return k * gridDim.x + pos;
+}
+
+// Map a linear item to (bh, q tile).  Non-causal: head-major, so CTAs running at
+// the same time share a head's K/V in L2.  Causal: heads are swept in groups;
+// inside a group the longest rows (highest q tile) come first.
+__device__ __forceinline__ void fwd_decode_item(const FwdParams& p, int w, int& bh, int& qt) {
+  if (!p.causal) {
+    bh = w / p.n_qt;
+    qt = w - bh * p.n_qt;
+    return;
+  }
+  const int per_group = p.group_heads * p.n_qt;
+  const int g = w / per_group;
+  const int r = w - g * per_group;
+  const int gsize = min(p.group_heads, p.BH - g * p.group_heads);
+  const int lvl = r / gsize;
+  qt = p.n_qt - 1 - lvl;
+  bh = g * p.group_heads + (r - lvl * gsize);
+}
+
+template <class C>
+__device__ __forceinline__ int fwd_num_kv_tiles(const FwdParams& p, int qt) {
+  if (!p.causal) return p.n_kt;
+  const int last = min(p.n_kt - 1, ((qt + 1) * C::BM - 1) / C::BN);
+  return last + 1;
+}
+
+// ---------------------------------------------------------------- producer (one thread)
+template <class C>
+__device__ void fwd_producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                             const FwdParams& p, uint32_t sbase, uint32_t bars, const WaitCtl& wc) {
+  auto bar = [&](int i) { return bars + 8u * i; };
+  uint32_t g = 0, t = 0;
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int w = fwd_item_index(k);
+    if (w >= p.total_items) break;
+    int bh, qt;
+    fwd_decode_item(p, w, bh, qt);
+    const int n = fwd_num_kv_tiles<C>(p, qt);
+    if (t > 0 && !(ok = mbar_wait(bar(C::B_QEMPTY), (t - 1) & 1, wc, kSiteQEmpty))) break;
+    mbar_arrive_expect_tx(bar(C::B_QFULL), C::Q_BYTES);
+#pragma unroll
+    for (int c = 0; c < C::NBOX; ++c)
+      tma_load_3d(sbase + C::SMEM_Q + c * C::BM * 128, tq, bar(C::B_QFULL), c * C::BOX_ELEMS,
+                  qt * C::BM, bh);
+    for (int j = 0; j < n; ++j) {
+      const uint32_t gj = g + j;
+      const int s = gj % C::STAGES;
+      if (gj >= C::STAGES &&
+          !(ok = mbar_wait(bar(C::B_KVEMPTY + s), ((gj / C::STAGES) - 1) & 1, wc, kSiteKVEmpty)))
+        break;
+      mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::KV_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::NBOX; ++c)
+        tma_load_3d(sbase + C::SMEM_K + s * C::KV_BYTES + c * C::BN * 128, tk,
+                    bar(C::B_KFULL + s), c * C::BOX_ELEMS, j * C::BN, bh);
+      mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::KV_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::NBOX; ++c)
+        tma_load_3d(sbase + C::SMEM_V + s * C::KV_BYTES + c * C::BN * 128, tv,
+                    bar(C::B_VFULL + s), c * C::BOX_ELEMS, j * C::BN, bh);
+    }
+    g += n;
+    ++t;
+  }
+  if (!ok) {
+    // Aborted: let the tile copies already issued land before the CTA exits.
+    if (t > 0 || g > 0) mbar_wait_drain(bar(C::B_QFULL), (t > 0 ? t - 1 : 0) & 1, 100000000ull);
+    for (uint32_t gk = (g > C::STAGES ? g - C::STAGES : 0); gk < g; ++gk) {
+      mbar_wait_drain(bar(C::B_KFULL + gk % C::STAGES), (gk / C::STAGES) & 1, 100000000ull);
+      mbar_wait_drain(bar(C::B_VFULL + gk % C::STAGES), (gk / C::STAGES) & 1, 100000000ull);
+    }
+    return;
+  }
+  // Drain: wait until the MMA side has released every buffer, so no tensor-core
+  // commit is still due to arrive on this CTA's barriers when it exits.
+  if (t > 0) {
+    ok = mbar_wait(bar(C::B_QEMPTY), (t - 1) & 1, wc, kSiteQEmpty);
+    for (uint32_t gk = (g > C::STAGES ? g - C::STAGES : 0); ok && gk < g; ++gk)
+      ok = mbar_wait(bar(C::B_KVEMPTY + gk % C::STAGES), (gk / C::STAGES) & 1, wc, kSiteKVEmpty);
+  }
+}
+
+// ---------------------------------------------------------------- MMA issuer (one thread)
+template <class C>
+__device__ void fwd_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                        const WaitCtl& wc) {
+  auto bar = [&](int i) { return bars + 8u * i; };
+  constexpr uint32_t IDESC_S = C::FP8 ? idesc_e4m3(128, C::BN, false) : idesc_bf16(128, C::BN, false);
+  constexpr uint32_t IDESC_O = C::FP8 ? idesc_e4m3(128, C::D, true) : idesc_bf16(128, C::D, true);
+  constexpr int KSTEPS_S = C::D / C::MMA_K;     // over the head dimension
+  constexpr int KSTEPS_O = C::BN / C::MMA_K;    // over the key tile
+  uint32_t g = 0, t = 0;
+  bool ok = true;
+
+  // O += P V for global step gk; `first` = first step of its item (overwrite O).
+  auto issue_pv = [&](uint32_t gk, bool first) -> bool {
+    const int b = gk & 1;
+    if (!mbar_wait(bar(C::B_PFULL + b), (gk >> 1) & 1, wc, kSitePFull)) return false;
+    const int s = gk % C::STAGES;
+    if (!mbar_wait(bar(C::B_VFULL + s), (gk / C::STAGES) & 1, wc, kSiteVFull)) return false;
+    tc_fence_after();
+    const uint32_t vbase = sbase + C::SMEM_V + s * C::KV_BYTES;
+#pragma unroll
+    for (int kb = 0; kb < KSTEPS_O; ++kb) {
+      // V tile is K(=key)-rows x N(=d) with d contiguous: MN-major operand.
+      // LBO = distance between 128-byte column boxes, SBO = 8 rows * 128 B.
+      const uint64_t bdesc = sdesc_sw128(vbase + kb * C::MMA_K * 128, C::BN * 128, 1024);
+      const uint32_t a_tmem = tmem + C::TM_S + b * C::BN + kb * (C::MMA_K * C::ELEM / 4);
+      umma_ts<C::FP8>(tmem + C::TM_O, a_tmem, bdesc, IDESC_O, (first && kb == 0) ? 0u : 1u);
+    }
+    tc_commit(bar(C::B_KVEMPTY + s));
+    tc_commit(bar(C::B_ODONE));
+    return true;
+  };
+
+  for (int k = 0; ok; ++k) {
+    const int w = fwd_item_index(k);
+    if (w >= p.total_items) break;
+    int bh, qt;
+    fwd_decode_item(p, w, bh, qt);
+    const int n = fwd_num_kv_tiles<C>(p, qt);
+    if (!(ok = mbar_wait(bar(C::B_QFULL), t & 1, wc, kSiteQFull))) break;
+    tc_fence_after();
+    for (int j = 0; j < n && ok; ++j) {
+      const uint32_t gj = g + j;
+      const int s = gj % C::STAGES;
+      if (!(ok = mbar_wait(bar(C::B_KFULL + s), (gj / C::STAGES) & 1, wc, kSiteKFull))) break;
+      tc_fence_after();
+      const int b = gj & 1;
+      const uint32_t kbase = sbase + C::SMEM_K + s * C::KV_BYTES;
+#pragma unroll
+      for (int kb = 0; kb < KSTEPS_S; ++kb) {
+        // K-major operands: 128-byte swizzled rows, 8-row groups 1024 B apart;
+        // a K step inside a 128-byte row is a 32-byte start-address offset.
+        const int box = (kb * C::KSTEP_BYTES) / 128;
+        const int off = (kb * C::KSTEP_BYTES) % 128;
+        const uint64_t adesc = sdesc_sw128(sbase + C::SMEM_Q + box * C::BM * 128 + off, 16, 1024);
+        const uint64_t bdesc = sdesc_sw128(kbase + box * C::BN * 128 + off, 16, 1024);
+        umma_ss<C::FP8>(tmem + C::TM_S + b * C::BN, adesc, bdesc, IDESC_S, kb > 0 ? 1u : 0u);
+      }
+      tc_commit(bar(C::B_SFULL + b));
+      if (j == n - 1) tc_commit(bar(C::B_QEMPTY));
+      if (j > 0) ok = issue_pv(gj - 1, j == 1);
+    }
+    if (ok) ok = issue_pv(g + n - 1, n == 1);
+    g += n;
+    ++t;
+  }
+  // Make sure nothing is in flight before the CTA frees tensor memory.
+  tc_commit(bar(C::B_DRAIN));
+  if (!mbar_wait_drain(bar(C::B_DRAIN), 0, wc.timeout_ns))
+    atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
+}
+
+// ---------------------------------------------------------------- softmax warps
+template <class C>
+__device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, const WaitCtl& wc) {
+  auto bar = [&](int i) { return bars + 8u * i; };
+  const int warp = threadIdx.x / 32;
+  const int quad = warp & 3;
+  const int row = quad * 32 + (threadIdx.x & 31);         // query row inside the tile
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+  const float LOG2E = 1.4426950408889634f;
+  const float LN2 = 0.6931471805599453f;
+  const float sl2 = p.scale * LOG2E;
+  __nv_bfloat16* o_out = reinterpret_cast<__nv_bfloat16*>(p.o);
+  uint32_t g = 0;
+  bool ok = true;
+
+  for (int k = 0; ok; ++k) {
+    const int w = fwd_item_index(k);
+    if (w >= p.total_items) break;
+    int bh, qt;
+    fwd_decode_item(p, w, bh, qt);
+    const int n = fwd_num_kv_tiles<C>(p, qt);
+    const int q_idx = qt * C::BM + row;
+    float m = -INFINITY, l = 0.f;
+    float qsc = 1.f, vmax = 1.f;
+    if constexpr (C::FP8) {
+      static_assert(!C::FP8 || C::BN == 128, "FP8 key tile = one 128-row scale tile");
+      qsc = p.q_scale[bh * p.n_st + qt];
+      // vmax = largest V tile scale among the visited key tiles; every thread reads
+      // the same few values (L1 broadcast), so no cross-warp barrier is needed.
+      vmax = 0.f;
+      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[bh * p.n_st + j]);
+    }
+
+    for (int j = 0; j < n; ++j) {
+      const uint32_t gj = g + j;
+      const int b = gj & 1;
+      if (!(ok = mbar_wait(bar(C::B_SFULL + b), (gj >> 1) & 1, wc, kSiteSFull))) break;
+      tc_fence_after();
+      float s[C::BN];
+#pragma unroll
+      for (int c = 0; c < C::BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + C::TM_S + b * C::BN + c, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(r[i]);
+      }
+      const int kv0 = j * C::BN;
+      const bool need_mask = (p.causal && kv0 + C::BN - 1 > qt * C::BM) || (kv0 + C::BN > p.N);
+      if (need_mask) {
+        const int lim = p.causal ? min(q_idx, p.N - 1) : p.N - 1;   // last visible key
+#pragma unroll
+        for (int c = 0; c < C::BN; ++c)
+          if (kv0 + c > lim) s[c] = -INFINITY;
+      }
+      float c_j = sl2;
+      float fold = 1.f;
+      if constexpr (C::FP8) {
+        c_j = sl2 * qsc * p.k_scale[bh * p.n_st + j];
+        fold = 256.f * p.v_scale[bh * p.n_st + j] / vmax;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < C::BN; ++c) mx = fmaxf(mx, s[c]);
+      const float m_new = fmaxf(m, mx * c_j);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = ex2(m - m_use);          // 0 on the first tile (m = -inf)
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < C::BN; ++c) {
+        s[c] = ex2(fmaf(s[c], c_j, -m_use));
+        sum += s[c];
+      }
+      l = l * alpha + sum;
+      // P -> tensor memory over the consumed S columns
+      if constexpr (C::FP8) {
+#pragma unroll
+        for (int c = 0; c < C::BN; c += 128) {
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            r[i] = pack_e4m3x4(s[c + 4 * i] * fold, s[c + 4 * i + 1] * fold,
+                               s[c + 4 * i + 2] * fold, s[c + 4 * i + 3] * fold);
+          tmem_st32(lane_base + C::TM_S + b * C::BN + c / 4, r);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < C::BN; c += 64) {
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = pack_bf16x2(s[c + 2 * i], s[c + 2 * i + 1]);
+          tmem_st32(lane_base + C::TM_S + b * C::BN + c / 2, r);
+        }
+      }
+      // The previous P V product must be complete before O is touched; waiting on
+      // every step also keeps this warp's view of the O barrier phase exact.
+      if (j > 0) {
+        if (!(ok = mbar_wait(bar(C::B_ODONE), (gj - 1) & 1, wc, kSiteODone))) break;
+        tc_fence_after();
+        const bool changed = m_new > m;
+        if (__any_sync(0xffffffffu, changed)) {
+#pragma unroll 1
+          for (int c = 0; c < C::D; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(lane_base + C::TM_O + c, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(lane_base + C::TM_O + c, r);
+          }
+        }
+      }
+      m = m_new;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PFULL + b));
+    }
+    if (!ok) break;
+    // epilogue: O / l -> bf16 -> global; row logsumexp
+    const uint32_t glast = g + n - 1;
+    if (!(ok = mbar_wait(bar(C::B_ODONE), glast & 1, wc, kSiteODone))) break;
+    tc_fence_after();
+    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / l;
+    const bool row_ok = q_idx < p.N;
+    __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * C::D;
+#pragma unroll 1
+    for (int c = 0; c < C::D; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(lane_base + C::TM_O + c, r);
+      tmem_ld_wait(r);
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      }
+    }
+    if (row_ok && p.lse != nullptr)
+      p.lse[static_cast<size_t>(bh) * p.N + q_idx] = (m + __log2f(l)) * LN2;
+    tc_fence_before();
+    g += n;
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tv, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  const uint32_t bars = sbase + C::SMEM_BAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
+  const int warp = threadIdx.x / 32;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NBARS; ++i) {
+      uint32_t cnt = 1;
+      if (i == C::B_PFULL || i == C::B_PFULL + 1) cnt = 128;
+      mbar_init(bars + 8u * i, cnt);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, p.status, p.timeout_ns};
+
+  if (warp == 0) {
+    if ((threadIdx.x & 31) == 0) fwd_producer<C>(&tq, &tk, &tv, p, sbase, bars, wc);
+  } else if (warp == 1) {
+    if ((threadIdx.x & 31) == 0) fwd_mma<C>(p, sbase, bars, tmem, wc);
+  } else {
+    fwd_softmax<C>(p, bars, tmem, wc);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_COLS);
+  }
+}
+
+}  // namespace fa

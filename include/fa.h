@@ -1,0 +1,149 @@
+/*
+ * fa.h — C ABI of libfa.so: exact scaled-dot-product attention on B200 (sm_100a).
+ *
+ * What is computed (every entry point): for every batch b and head h,
+ *
+ *     O = softmax(Q K^T * scale) V
+ *
+ * "FlashAttention — フラッシュアテンション" (systems-analysis.info wiki), section
+ * 標準的なアテンションの問題点, displayed formula.  The work is done by fused,
+ * tiled kernels that never write the N x N score matrix to global memory
+ * (same page, sections タイリングとブロック処理 and CUDAカーネルの融合), with an
+ * online softmax that carries a running row max and row sum
+ * ("FlashAttentionとは？…" (issoh.co.jp), section 最大値と正規化項を持ち回る
+ * オンラインsoftmaxの再スケール).  Results equal the definition up to
+ * floating-point rounding, not bit for bit.
+ *
+ * Conventions shared by all entry points
+ * --------------------------------------
+ *  Layout    Q, K, V, O, dO, dQ, dK, dV are dense row-major [B, H, N, d]
+ *            (d contiguous, then N, then H, then B); LSE and the FP8 scales
+ *            are dense [B, H, N] and [B, H, ceil(N/128)].
+ *  Pointers  device pointers (cudaMalloc / torch CUDA memory) on the current
+ *            device, 16-byte aligned.  The caller owns every buffer; the
+ *            library allocates and frees no device memory on any call.
+ *  Sizes     B, H, N >= 0; d in {64, 128, 256} (bf16) or {128} (FP8).  N need
+ *            not be a multiple of 128.  A call with B*H*N == 0 returns FA_OK
+ *            and launches nothing (pointers may then be NULL).
+ *  causal    0 = every key visible; 1 = key j visible to query i iff j <= i
+ *            (lower triangular, top-left aligned; N_q == N_k).
+ *  scale     multiplier of Q K^T, finite and > 0 (SDPA's default is 1/sqrt(d)).
+ *  Streams   every call is asynchronous on `stream` (a cudaStream_t, 0 = the
+ *            legacy default stream) and never synchronises the host.
+ *  Errors    argument errors return at once, before any CUDA call, and launch
+ *            nothing.  There is no fallback path: an unsupported request fails
+ *            (issoh.co.jp page, section CPUのPyTorch SDPA…: a forced fused path
+ *            raises rather than silently running a slower one).
+ *            fa_last_error_string() describes the most recent failure of the
+ *            calling host thread.
+ *  Device    every spin-wait inside the kernels is bounded in time; on expiry
+ *            the kernel records a code in a device status word, drains its own
+ *            in-flight work, frees its tensor memory and exits.  Read it with
+ *            fa_get_device_status().
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,     /* NULL pointer, negative size, misalignment, bad scale */
+  FA_ERR_UNSUPPORTED = 2,     /* valid request outside what the kernels implement (d) */
+  FA_ERR_CUDA = 3,            /* a CUDA runtime call or kernel launch failed */
+  FA_ERR_DEVICE_TIMEOUT = 4   /* reported by fa_get_device_status: a bounded wait expired */
+} fa_status;
+
+/*
+ * fa_fwd — bf16 forward.  Tiled fused kernel: TMA tile loads, tcgen05 MMAs for
+ * S = Q K^T and O += P V with fp32 accumulators in tensor memory, exp2-based
+ * online softmax that rescales O only when a row max changes, causal tiles
+ * above the diagonal skipped, persistent heaviest-first tile scheduler.
+ *   q, k, v  in   bf16 [B,H,N,d]
+ *   o        out  bf16 [B,H,N,d]  = softmax(scale Q K^T) V, rounded to nearest even
+ *   lse      out  fp32 [B,H,N]    row logsumexp, natural log:
+ *                                  lse_i = ln sum_{j visible} exp(scale q_i . k_j)
+ *                                  (the normalisation statistic the backward reuses;
+ *                                  issoh.co.jp page, section 逆伝播でL×L行列を保存せず
+ *                                  再計算する設計).  May be NULL if not wanted.
+ * Returns FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED (d not 64/128/256) or FA_ERR_CUDA.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
+ * fa_fwd_fp8 — FP8 (e4m3, OCP "fn" variant) forward with per-tile scales
+ * (mypcrig.com post, section "FA3 の飛躍": per-tile rescaling and block-wise
+ * quantisation keep FP8 attention accurate).
+ *   q8, k8, v8        in  e4m3 [B,H,N,d]; real value = code * scale of its tile
+ *   q_scale, k_scale,
+ *   v_scale           in  fp32 [B,H,ceil(N/128)]: one scale per 128 consecutive rows
+ *   o                 out bf16 [B,H,N,d]; lse out fp32 [B,H,N] (may be NULL)
+ * The probabilities are rounded to e4m3 before the P V product (the product runs
+ * on the FP8 tensor cores); everything else accumulates in fp32.
+ * d must be 128.  Errors as fa_fwd.
+ */
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                     const float* q_scale, const float* k_scale, const float* v_scale,
+                     void* o, float* lse,
+                     int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
+ * fa_bwd_workspace_size — bytes of device workspace fa_bwd needs for these sizes
+ * (fp32 D_i = sum_c dO_ic O_ic for every row, 256-byte aligned).  0 when B*H*N == 0.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_bwd — bf16 backward by recomputation: the score tile is recomputed from
+ * Q and K, P is rebuilt from the saved lse, and no N x N matrix is stored
+ * (issoh.co.jp page, section 逆伝播でL×L行列を保存せず再計算する設計).
+ * Gradients of L = sum(O * dO):
+ *   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,  dS = P * (dP - D),
+ *   dQ = scale dS K,  dK = scale dS^T Q.
+ *   q, k, v, o, dO   in  bf16 [B,H,N,d] (o = fa_fwd's output for the same inputs)
+ *   lse              in  fp32 [B,H,N]   (fa_fwd's lse for the same inputs)
+ *   dq, dk, dv       out bf16 [B,H,N,d]
+ *   workspace        scratch device memory of >= fa_bwd_workspace_size() bytes,
+ *                    owned by the caller; contents on entry are ignored.
+ * Launches, in stream order: the D_i row-sum pass, the dK/dV pass (one CTA per
+ * key tile) and the dQ pass (one CTA per query tile).  Deterministic: no
+ * atomics.  Errors as fa_fwd, plus FA_ERR_INVALID_ARG when the workspace is
+ * too small.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes,
+                 int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/* fa_last_error_string — text of the calling thread's last failure ("" if none). */
+const char* fa_last_error_string(void);
+
+/*
+ * fa_get_device_status — synchronises `stream`, then reads and clears the
+ * device status word of the current device.  *code = 0 when no kernel has
+ * reported a problem; otherwise (FA_ERR_DEVICE_TIMEOUT << 24) | site, where
+ * site names the wait that expired.  Returns FA_ERR_CUDA if the copy fails.
+ */
+fa_status fa_get_device_status(void* stream, int* code);
+
+/*
+ * fa_debug_wait_timeout_selftest — launches one CTA that waits on a barrier
+ * nothing will ever complete, with the given bound in microseconds (1..2000000).
+ * The wait must expire, record FA_ERR_DEVICE_TIMEOUT in the status word and
+ * return; the context stays usable.  Used by the tests of the fault path.
+ */
+fa_status fa_debug_wait_timeout_selftest(int timeout_us, void* stream);
+
+/* fa_version — library version, major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FA_H_ */

@@ -1,0 +1,75 @@
+"""Shared comparison helpers and tolerances for the GPU-vs-oracle parity tests.
+
+Tolerances (stated once, used everywhere):
+  bf16 forward : O max |err| <= 1e-2, O mean |err| <= 1e-3, LSE max relative err <= 1e-3
+  bf16 backward: relative Frobenius error <= 2e-2 for each of dQ, dK, dV
+  FP8 forward  : O max |err| <= 6e-2 (against the oracle on the dequantised inputs)
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+O_MAX_ABS = 1e-2
+O_MEAN_ABS = 1e-3
+LSE_REL = 1e-3
+GRAD_REL_FRO = 2e-2
+FP8_O_MAX_ABS = 6e-2
+
+
+def to64(t) -> np.ndarray:
+    if isinstance(t, torch.Tensor):
+        return t.detach().float().cpu().double().numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+def fwd_errors(o, lse, o_ref, lse_ref) -> dict:
+    o, lse = to64(o), to64(lse)
+    e = np.abs(o - o_ref)
+    return {
+        "o_max_abs": float(e.max()) if e.size else 0.0,
+        "o_mean_abs": float(e.mean()) if e.size else 0.0,
+        "lse_max_rel": float((np.abs(lse - lse_ref) / np.maximum(np.abs(lse_ref), 1e-30)).max())
+        if lse.size else 0.0,
+        "lse_max_abs": float(np.abs(lse - lse_ref).max()) if lse.size else 0.0,
+    }
+
+
+def assert_fwd_ok(o, lse, o_ref, lse_ref, tag=""):
+    err = fwd_errors(o, lse, o_ref, lse_ref)
+    assert err["o_max_abs"] <= O_MAX_ABS, (tag, err)
+    assert err["o_mean_abs"] <= O_MEAN_ABS, (tag, err)
+    # LSE relative error: the pages' reading is "relative"; near LSE = 0 (causal row 0
+    # with q0.k0 ~ 0) a relative bound is meaningless, so small |LSE| use an absolute 1e-3.
+    lse_, ref_ = to64(lse), np.asarray(lse_ref)
+    bad = np.abs(lse_ - ref_) > LSE_REL * np.maximum(np.abs(ref_), 1.0)
+    assert not bad.any(), (tag, err, int(bad.sum()))
+    return err
+
+
+def rel_fro(g, ref) -> float:
+    g, ref = to64(g), np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref.ravel())
+    return float(np.linalg.norm((g - ref).ravel()) / max(den, 1e-30))
+
+
+def assert_grads_ok(got, ref, tag=""):
+    errs = {n: rel_fro(g, r) for n, g, r in zip(("dq", "dk", "dv"), got, ref)}
+    for n, e in errs.items():
+        assert e <= GRAD_REL_FRO, (tag, errs)
+    return errs
+
+
+def sample_rows(B, H, N, n_heads=4, n_rows=24, seed=0, extra_rows=()):
+    """(b, h, i) triples: tile edges, first/last rows and random rows of a few heads."""
+    rng = np.random.default_rng(seed)
+    heads = {(0, 0), (B - 1, H - 1)}
+    while len(heads) < min(n_heads, B * H):
+        heads.add((int(rng.integers(B)), int(rng.integers(H))))
+    fixed = {0, 1, 127, 128, 129, N // 2, N - 129, N - 128, N - 2, N - 1, *extra_rows}
+    out = []
+    for b, h in sorted(heads):
+        rows = {r for r in fixed if 0 <= r < N}
+        rows |= set(rng.integers(0, N, size=n_rows).tolist())
+        out += [(b, h, r) for r in sorted(rows)]
+    return np.array(out, dtype=np.int64)

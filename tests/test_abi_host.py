@@ -1,0 +1,91 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+symbol include/fa.h declares, and rejects bad arguments before any CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import exact_attention_132_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_size",
+                     "fa_last_error_string", "fa_get_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (fa_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(fa.lib, n)
+
+
+def test_version():
+    assert fa.fa_version() >= 100
+
+
+def _fwd(q=1, k=1, v=1, o=1, lse=None, B=1, H=1, N=128, d=128, scale=0.1, causal=0):
+    P = lambda x: None if x is None else ctypes.c_void_p(16 * x)
+    return fa.lib.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, scale, causal, None)
+
+
+def test_argument_errors_return_before_any_cuda_call():
+    assert _fwd(q=None) == fa.FA_ERR_INVALID_ARG
+    assert "q is NULL" in fa.fa_last_error_string()
+    assert _fwd(B=-1) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(scale=0.0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(scale=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(scale=-1.0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(d=32) == fa.FA_ERR_UNSUPPORTED
+    # misaligned pointer
+    assert fa.lib.fa_fwd(ctypes.c_void_p(18), ctypes.c_void_p(16), ctypes.c_void_p(16),
+                         ctypes.c_void_p(16), None, 1, 1, 128, 64, 0.1, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert "aligned" in fa.fa_last_error_string()
+
+
+def test_empty_problems_are_a_no_op():
+    assert _fwd(q=None, k=None, v=None, o=None, N=0) == fa.FA_OK
+    assert _fwd(q=None, k=None, v=None, o=None, B=0) == fa.FA_OK
+    assert fa.lib.fa_bwd(None, None, None, None, None, None, None, None, None, None, 0,
+                         1, 4, 0, 64, 0.125, 1, None) == fa.FA_OK
+    assert fa.fa_bwd_workspace_size(0, 4, 128, 64) == 0
+
+
+def test_fp8_and_bwd_argument_errors():
+    P = lambda x: ctypes.c_void_p(16 * x)
+    st = fa.lib.fa_fwd_fp8(P(1), P(1), P(1), None, P(1), P(1), P(1), None, 1, 1, 256, 128, 0.1, 1, None)
+    assert st == fa.FA_ERR_INVALID_ARG
+    st = fa.lib.fa_fwd_fp8(P(1), P(1), P(1), P(1), P(1), P(1), P(1), None, 1, 1, 256, 64, 0.1, 1, None)
+    assert st == fa.FA_ERR_UNSUPPORTED
+    need = fa.fa_bwd_workspace_size(2, 3, 1000, 64)
+    assert need >= 2 * 3 * 1000 * 4 and need % 256 == 0
+    st = fa.lib.fa_bwd(P(1), P(1), P(1), P(1), P(1), P(1), P(1), P(1), P(1), P(1), need - 256,
+                       2, 3, 1000, 64, 0.125, 0, None)
+    assert st == fa.FA_ERR_INVALID_ARG and "workspace" in fa.fa_last_error_string()
+
+
+def test_python_wrappers_validate_shapes():
+    import torch
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        fa.fa_fwd(q.float(), q, q, q)
+    with pytest.raises(ValueError):
+        fa.fa_fwd(q, q[:, :1], q, q)
+    with pytest.raises(ValueError):
+        fa.fa_fwd(q, q, q, q)   # CPU tensors are rejected: no CPU path exists

@@ -1,0 +1,102 @@
+"""bf16 forward: CUDA path (through the C ABI) vs the fp64 oracle on the same inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fa():
+    import exact_attention_132_b200 as m
+    return m
+
+
+SMALL = [
+    # (B, H, N, d, causal)  several tiles, ragged tails, every head dim
+    (1, 2, 128, 64, False), (1, 2, 128, 64, True),
+    (2, 3, 513, 64, True), (2, 2, 700, 64, False),
+    (1, 3, 384, 128, True), (2, 2, 1000, 128, False), (1, 2, 1000, 128, True),
+    (1, 2, 320, 256, True), (1, 2, 520, 256, False),
+    (1, 1, 1, 64, True), (1, 1, 77, 128, False),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", SMALL)
+def test_fwd_small_matches_oracle(fa, B, H, N, d, causal):
+    w = workloads.make_small(B, H, N, d, causal, seed=N * 7 + d, backward=False)
+    q, k, v = workloads.make_bf16_inputs(w)
+    o, lse = fa.attention_forward(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=w.sm_scale)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attention_fwd(q, k, v, w.sm_scale, causal)
+    parity.assert_fwd_ok(o, lse, o_ref, lse_ref, tag=w.name)
+    assert fa.fa_get_device_status() == 0
+
+
+def test_fwd_small_workload_full(fa):
+    """B=1 H=8 N=1024 d=64 causal, scale 1/8: every output element checked."""
+    w = workloads.WORKLOADS["fwd_small"]
+    q, k, v = workloads.make_bf16_inputs(w)
+    o, lse = fa.attention_forward(q.cuda(), k.cuda(), v.cuda(), causal=True, scale=w.sm_scale)
+    o_ref, lse_ref = oracle.attention_fwd(q, k, v, w.sm_scale, True)
+    err = parity.assert_fwd_ok(o, lse, o_ref, lse_ref, tag=w.name)
+    print("fwd_small", err)
+
+
+def test_fwd_outlier_workload_full_size_sampled(fa):
+    """B=4 H=16 N=4096 d=128 causal with 1% K outlier rows, run at full size in the
+    benchmark's launch configuration; sampled rows are checked one by one against the
+    oracle (each sampled row still sees all of its keys)."""
+    w = workloads.WORKLOADS["fwd_d128"]
+    q, k, v = workloads.make_bf16_inputs(w)
+    o, lse = fa.attention_forward(q.cuda(), k.cuda(), v.cuda(), causal=True, scale=w.sm_scale)
+    picks = parity.sample_rows(w.B, w.H, w.N, n_heads=6, n_rows=40, seed=2)
+    o_ref, lse_ref = oracle.attention_fwd_rows(q, k, v, w.sm_scale, True, picks)
+    og, lg = o.cpu(), lse.cpu()
+    got_o = np.stack([parity.to64(og[b, h, i]) for b, h, i in picks])
+    got_l = np.array([float(lg[b, h, i]) for b, h, i in picks])
+    err = parity.assert_fwd_ok(got_o, got_l, o_ref, lse_ref, tag=w.name)
+    print("fwd_d128 sampled", err)
+    # whole-output properties that hold at any size
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    # causal row 0 of every head is V_0 exactly (a single visible key) and LSE_0 = scale q0.k0
+    assert torch.equal(o[:, :, 0].cpu(), v[:, :, 0])
+    ref_l0 = (q[:, :, 0].double() * k[:, :, 0].double()).sum(-1) * w.sm_scale
+    assert (lse[:, :, 0].cpu().double() - ref_l0).abs().max() < 1e-3 * max(1.0, ref_l0.abs().max())
+
+
+def test_fwd_is_deterministic(fa):
+    w = workloads.make_small(2, 4, 1024, 128, True, seed=3, backward=False)
+    q, k, v = (t.cuda() for t in workloads.make_bf16_inputs(w))
+    o1, l1 = fa.attention_forward(q, k, v, causal=True)
+    o2, l2 = fa.attention_forward(q, k, v, causal=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fwd_on_side_stream_and_lse_optional(fa):
+    w = workloads.make_small(1, 2, 256, 64, False, seed=5, backward=False)
+    q, k, v = (t.cuda() for t in workloads.make_bf16_inputs(w))
+    s = torch.cuda.Stream()
+    o = torch.empty_like(q)
+    with torch.cuda.stream(s):
+        fa.fa_fwd(q, k, v, o, None, causal=False)
+    s.synchronize()
+    o_ref, _ = oracle.attention_fwd(q.cpu(), k.cpu(), v.cpu(), w.sm_scale, False)
+    assert np.abs(parity.to64(o) - o_ref).max() <= parity.O_MAX_ABS
+
+
+def test_unsupported_head_dim_raises(fa):
+    q = torch.zeros(1, 1, 128, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fa.FAError) as ei:
+        fa.attention_forward(q, q, q)
+    assert ei.value.status == fa.FA_ERR_UNSUPPORTED
+
+
+def test_empty_sequence_is_a_no_op(fa):
+    q = torch.zeros(2, 3, 0, 64, dtype=torch.bfloat16, device="cuda")
+    o, lse = fa.attention_forward(q, q, q, causal=True)
+    assert o.shape == (2, 3, 0, 64) and lse.shape == (2, 3, 0)
