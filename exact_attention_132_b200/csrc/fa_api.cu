@@ -103,8 +103,9 @@ fa_status make_map(CUtensorMap* m, const void* ptr, bool fp8, int d, int N, int 
   return FA_OK;
 }
 
-// Set the dynamic shared-memory limit of a kernel once per device.
-template <class K>
+// Set the dynamic shared-memory limit of a kernel once per device.  `Tag` makes the
+// cache per kernel: every kernel here has the same signature, so K alone does not.
+template <class Tag, class K>
 fa_status prepare_kernel(K kernel, int smem_bytes) {
   static std::atomic<uint64_t> done{0};
   int dev = 0;
@@ -154,7 +155,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, FwdParams p, c
   if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
   if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
   auto kern = fa_fwd_kernel<C>;
-  if (fa_status s = prepare_kernel(kern, C::SMEM_ALLOC)) return s;
+  if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
   p.n_qt = (p.N + C::BM - 1) / C::BM;
   p.n_kt = (p.N + C::BN - 1) / C::BN;
   p.n_st = (p.N + 127) / 128;
@@ -210,7 +211,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH, CK::BN)) return s;
     if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH, CK::BN)) return s;
     auto kern = fa_bwd_dkdv<CK>;
-    if (fa_status s = prepare_kernel(kern, CK::SMEM_ALLOC)) return s;
+    if (fa_status s = prepare_kernel<CK>(kern, CK::SMEM_ALLOC)) return s;
     BwdParams pk = p;
     pk.n_qt = (p.N + CK::BMQ - 1) / CK::BMQ;
     pk.n_kt = (p.N + CK::BN - 1) / CK::BN;
@@ -227,7 +228,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH, CQ::BN)) return s;
     if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH, CQ::BN)) return s;
     auto kern = fa_bwd_dq<CQ>;
-    if (fa_status s = prepare_kernel(kern, CQ::SMEM_ALLOC)) return s;
+    if (fa_status s = prepare_kernel<CQ>(kern, CQ::SMEM_ALLOC)) return s;
     BwdParams pq = p;
     pq.n_qt = (p.N + CQ::BM - 1) / CQ::BM;
     pq.n_kt = (p.N + CQ::BN - 1) / CQ::BN;
