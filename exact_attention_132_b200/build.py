@@ -1,6 +1,6 @@
 """Build libfa.so (the C-ABI attention library) in-tree with nvcc for sm_100a.
 
-    python -m exact_attention_132_b200.build [--verbose] [--ptxas-info]
+    python exact_attention_132_b200/build.py [--verbose] [--ptxas-info]
 
 The shared library lands next to this file; the Python binding loads it from
 there.  The CUDA runtime is linked statically, so the library needs only the
