@@ -5,7 +5,7 @@ device pointers and the current CUDA stream from torch, and calls the C entry
 point of the same name (declared in include/fa.h).  All arithmetic runs in the
 library's CUDA kernels; there is no Python or CPU fallback, and importing this
 package fails if the library has not been built
-(``python -m exact_attention_132_b200.build``).
+(``python exact_attention_132_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -37,7 +37,7 @@ class FAError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m exact_attention_132_b200.build`")
+                          "`python exact_attention_132_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     L.fa_bwd_workspace_size.restype = sz
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
+    L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    L.fa_bwd_noalloc.restype = ctypes.c_int
     L.fa_last_error_string.argtypes = []
     L.fa_last_error_string.restype = ctypes.c_char_p
     L.fa_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
@@ -148,6 +150,26 @@ def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, scale: float | None = Non
     _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk),
                       _ptr(dv), _ptr(workspace), ws_bytes, B, H, N, d, sc, 1 if causal else 0,
                       _stream(stream)))
+
+
+FA_BWD_NOALLOC_MAX_ROWS = 1 << 21
+
+
+def fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, scale: float | None = None,
+                   causal: bool = False, stream=None):
+    """fa_bwd without a workspace argument, for callers that cannot allocate device
+    memory: the library uses its own fixed scratch (B*H*N <= FA_BWD_NOALLOC_MAX_ROWS).
+    Calls that overlap on the GPU share that scratch and race; serialise them."""
+    B, H, N, d = _bhnd(q, "q", torch.bfloat16)
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (dO, "dO"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if _bhnd(t, n, torch.bfloat16) != (B, H, N, d):
+            raise ValueError(f"{n} shape differs from q")
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be fp32 [B, H, N]")
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq),
+                              _ptr(dk), _ptr(dv), B, H, N, d, sc, 1 if causal else 0,
+                              _stream(stream)))
 
 
 def fa_get_device_status(stream=None) -> int:

@@ -260,6 +260,36 @@ size_t workspace_bytes(int B, int H, int N) {
   return (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
 }
 
+// ------------------------------------------------------------------ no-allocation backward
+// Fixed scratch for fa_bwd_noalloc: one fp32 D_i per row (B*H*N rows at most
+// FA_BWD_NOALLOC_MAX_ROWS).  It lives in the module image, so every GPU that loads
+// this library holds these 8 MiB until the process exits.  In host code the name
+// is only a host-side stand-in; kernels get the device address looked up below.
+static __device__ __align__(256) float g_bwd_noalloc_scratch[FA_BWD_NOALLOC_MAX_ROWS];
+
+struct NoallocScratch {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  float* ptr = nullptr;
+};
+NoallocScratch g_noalloc[kMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once per
+// device with that device current.
+fa_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_CUDA, "device index %d out of range", dev);
+  NoallocScratch& s = g_noalloc[dev];
+  std::call_once(s.once, [&] {
+    s.err = cudaGetSymbolAddress(reinterpret_cast<void**>(&s.ptr), g_bwd_noalloc_scratch);
+  });
+  if (s.err != cudaSuccess) return cuda_fail(s.err, "cudaGetSymbolAddress(no-alloc scratch)");
+  *out = s.ptr;
+  return FA_OK;
+}
+
 }  // namespace fa
 
 using namespace fa;
@@ -348,6 +378,48 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.scale = scale;
   p.lse = lse;
   p.drow = static_cast<const float*>(workspace);
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_bwd<DkdvD64, DqD64>(q, k, v, o, dO, p, st);
+    case 128: return launch_bwd<DkdvD128, DqD128>(q, k, v, o, dO, p, st);
+    default: return launch_bwd<DkdvD256, DqD256>(q, k, v, o, dO, p, st);
+  }
+}
+
+// Same kernels and results as fa_bwd, but the per-row D_i scratch comes from the
+// library's own fixed device array instead of a caller workspace, so this call
+// never allocates.  The first call on a device looks up the array's address
+// (cudaGetSymbolAddress) with that device current.  D_i is fully rewritten before
+// it is read, so nothing needs clearing between calls; calls that overlap on the
+// GPU (other streams, other threads) share the array and race.
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                         float scale, int causal, void* stream) {
+  bool empty = false;
+  if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
+  if (d != 64 && d != 128 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
+  if (empty) return FA_OK;
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (rows > FA_BWD_NOALLOC_MAX_ROWS)
+    return fail(FA_ERR_INVALID_ARG,
+                "fa_bwd_noalloc: B*H*N = %lld rows exceeds the fixed scratch of %d rows; "
+                "use fa_bwd with a caller workspace", rows, FA_BWD_NOALLOC_MAX_ROWS);
+  const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
+  const char* names[] = {"q", "k", "v", "o", "dO", "lse", "dq", "dk", "dv"};
+  if (fa_status s = check_ptrs(ptrs, names, 9)) return s;
+  float* scratch = nullptr;
+  if (fa_status s = noalloc_scratch(&scratch)) return s;
+  BwdParams p{};
+  p.BH = B * H;
+  p.N = N;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.lse = lse;
+  p.drow = scratch;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;

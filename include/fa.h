@@ -121,6 +121,33 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* workspace, size_t workspace_bytes,
                  int B, int H, int N, int d, float scale, int causal, void* stream);
 
+/*
+ * fa_bwd_noalloc — fa_bwd for callers that cannot allocate device memory.
+ * (The pages describe nothing like it; it exists for integration only.)
+ * Some callers have no way to hand the library a workspace: a plugin inside a
+ * host program that owns every byte of device memory through its own pool, or a
+ * latency-critical path where cudaMalloc's implicit device-wide synchronisation
+ * is not acceptable.  This entry point takes the same inputs and outputs as
+ * fa_bwd and gives the same results, but keeps the per-row D_i scratch in a fixed
+ * array inside the library (FA_BWD_NOALLOC_MAX_ROWS fp32 values = 8 MiB, held on
+ * every GPU that loads the library until the process exits).  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *   Sizes: B*H*N must be <= FA_BWD_NOALLOC_MAX_ROWS, else FA_ERR_INVALID_ARG
+ *          (use fa_bwd with a caller workspace for larger problems).
+ *   Set-up: the first call on each device looks up the array's device address
+ *          with that device current; make that first call before any stream
+ *          capture.
+ *   Sharing: all calls on a device share the one array.  D_i is fully rewritten
+ *          by each call before it is read, so no clearing is needed, but calls
+ *          that overlap on the GPU (other streams or host threads) race and give
+ *          wrong gradients: serialise them.
+ * Other arguments and errors as fa_bwd.
+ */
+#define FA_BWD_NOALLOC_MAX_ROWS (1 << 21)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                         int B, int H, int N, int d, float scale, int causal, void* stream);
+
 /* fa_last_error_string — text of the calling thread's last failure ("" if none). */
 const char* fa_last_error_string(void);
 
