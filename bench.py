@@ -42,9 +42,21 @@ METRIC = "attention TFLOP/s fwd and fwd+bwd on 1 B200; % of dense BF16/FP8 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per launch of the forward kernel at the headline workload,
-# from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` (profiles/
-# fa_fwd_d128_causal_B4H16N4096.md).  None until a capture of the current kernel exists.
-FWD_TRAFFIC_BYTES = None
+# from ncu's dram__bytes_read.sum + dram__bytes_write.sum (profiles/
+# fa_fwd_d128_causal_B4H16N4096.md), keyed by the hash of the kernel sources they were
+# measured on.  A changed kernel has no entry and reports traffic = null.
+FWD_TRAFFIC_BYTES = {"785b081eb6926ca8": 279_987_456}
+KERNEL_SOURCES = ("exact_attention_132_b200/csrc/fa_fwd.cuh",
+                  "exact_attention_132_b200/csrc/sm100_ptx.cuh")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    parts = []
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            parts.append(hashlib.sha256(f.read()).hexdigest() + "\n")
+    return hashlib.sha256("".join(parts).encode()).hexdigest()[:16]
 
 
 # ------------------------------------------------------------------ helpers
@@ -140,6 +152,7 @@ def time_steps(fn, steps, warmup, stream):
 # ------------------------------------------------------------------ our implementation
 def run_ours(args):
     import exact_attention_132_b200 as fa
+    from exact_attention_132_b200.multi_gpu import aggregate_throughput
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -168,13 +181,10 @@ def run_ours(args):
     clocks.start()
     total_ms, per = time_steps(step, args.steps, args.warmup, stream)
     clk = clocks.stop()
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        dist.barrier()
     flops = w.fwd_flops()
-    value = flops * args.steps * world / (total_ms * 1e-3) / 1e12
+    value, total_ms = aggregate_throughput(flops, args.steps, total_ms, dist, dev)
+    if dist is not None:
+        dist.barrier()
     kernel_ms = statistics.mean(per)
     achieved = flops / (kernel_ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
@@ -196,11 +206,7 @@ def run_ours(args):
 
     e2e_steps = max(3, min(args.steps, 10))
     e2e_ms, _ = time_steps(e2e_step, e2e_steps, 2, stream)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_val, e2e_ms = aggregate_throughput(flops, e2e_steps, e2e_ms, dist, dev)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
 
@@ -235,7 +241,8 @@ def run_ours(args):
                      "peak_source": f"{peak_src} bf16 dense matmul (burst)",
                      "kernel": "fa_fwd_kernel<FwdCfg<128,128,2,false>>",
                      "kernel_ms": round(kernel_ms, 4),
-                     "traffic": FWD_TRAFFIC_BYTES},
+                     "traffic": FWD_TRAFFIC_BYTES.get(kernel_source_hash()),
+                     "kernel_source_hash": kernel_source_hash()},
         "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "ms_per_step": round(e2e_ms / e2e_steps, 4)},
@@ -376,8 +383,38 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_driver(name, launches):
+    """Launch one workload's kernels a few times and exit: the target for ncu captures
+    (`ncu -k regex:... -s <skip> -c <n> python bench.py --profile <name>`)."""
+    import exact_attention_132_b200 as fa
+    w = workloads.WORKLOADS[name]
+    dev = torch.device("cuda", 0)
+    if w.fp8:
+        inp = workloads.make_fp8_inputs(w)
+        t = {n: inp[n].to(dev) for n in ("q8", "k8", "v8", "qs", "ks", "vs")}
+        o = torch.empty(t["q8"].shape, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(t["q8"].shape[:3], dtype=torch.float32, device=dev)
+        for _ in range(launches):
+            fa.fa_fwd_fp8(t["q8"], t["k8"], t["v8"], t["qs"], t["ks"], t["vs"], o, lse,
+                          scale=w.sm_scale, causal=w.causal)
+    else:
+        ins = [x.to(dev) for x in workloads.make_bf16_inputs(w)]
+        q, k, v = ins[:3]
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        for _ in range(launches):
+            fa.fa_fwd(q, k, v, o, lse, scale=w.sm_scale, causal=w.causal)
+            if w.backward:
+                fa.attention_backward(q, k, v, o, ins[3], lse, causal=w.causal, scale=w.sm_scale)
+    torch.cuda.synchronize()
+    print(f"profile driver {name}: {launches} launches, status {fa.fa_get_device_status()}")
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile", choices=sorted(workloads.WORKLOADS), default=None,
+                    help="only launch this workload's kernels (--profile-launches times) for ncu")
+    ap.add_argument("--profile-launches", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
@@ -389,7 +426,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile:
+        run_profile_driver(args.profile, args.profile_launches)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
