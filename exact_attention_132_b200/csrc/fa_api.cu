@@ -170,10 +170,20 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, FwdParams p, c
   return FA_OK;
 }
 
-using FwdD64 = FwdCfg<64, 128, 3, false>;
-using FwdD128 = FwdCfg<128, 128, 2, false>;
-using FwdD256 = FwdCfg<256, 64, 2, false>;
-using FwdF8D128 = FwdCfg<128, 128, 3, true>;
+// Tuning knobs (compile-time): software-exp2 share and pipeline depth.
+#ifndef FA_FWD_EMU
+#define FA_FWD_EMU 1
+#endif
+#ifndef FA_FWD_D128_KST
+#define FA_FWD_D128_KST 3
+#endif
+#ifndef FA_FWD_D128_VST
+#define FA_FWD_D128_VST 2
+#endif
+using FwdD64 = FwdCfg<64, 128, 4, 4, false, FA_FWD_EMU>;
+using FwdD128 = FwdCfg<128, 128, FA_FWD_D128_KST, FA_FWD_D128_VST, false, FA_FWD_EMU>;
+using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_EMU>;
+using FwdF8D128 = FwdCfg<128, 128, 4, 4, true, FA_FWD_EMU>;
 
 using DkdvD64 = DkdvCfg<64, 64, 128, 3>;
 using DkdvD128 = DkdvCfg<128, 128, 128, 2>;

@@ -20,7 +20,7 @@
 // never visited (mypcrig.com post, section "FA2 の改善").
 //
 // Roles (warp specialisation, mypcrig.com post, section "FA3 の飛躍"):
-//   warp 0       TMA producer: Q tile per item, K/V tiles into a STAGES-deep ring
+//   warp 0       TMA producer: Q tile per item, K and V tiles into separate rings
 //   warp 1       MMA issuer (one thread) + tensor-memory owner
 //   warps 2..5   softmax/correction/epilogue: thread t owns query row 32*(w%4)+lane,
 //                which is TMEM lane 32*(w%4)+lane (the lane quadrant a warp may use)
@@ -30,6 +30,8 @@
 //   [BN, 2BN)    S buffer 1
 //   [2BN, 2BN+D) O accumulator (fp32)
 #pragma once
+
+#include <type_traits>
 
 #include "sm100_ptx.cuh"
 
@@ -54,12 +56,23 @@ struct FwdParams {
   unsigned long long timeout_ns;
 };
 
-template <int D_, int BN_, int STAGES_, bool FP8_>
+template <int D_, int BN_, int KST_, int VST_, bool FP8_, int EMU_ = 1>
 struct FwdCfg {
   static constexpr int D = D_;
   static constexpr int BN = BN_;
-  static constexpr int STAGES = STAGES_;
+  // Separate K and V rings: a K stage is released as soon as its S = Q K^T product
+  // completes, a V stage when its P V product completes.
+  static constexpr int KST = KST_;
+  static constexpr int VST = VST_;
   static constexpr bool FP8 = FP8_;
+  // Of every 4 column pairs of a score row, EMU take their exponentials on the FMA
+  // pipe (ex2_poly_pair), the rest on the special-function unit.
+  static constexpr int EMU = EMU_;
+  // Reference-max slack in log2 units: the running max used for the exponentials
+  // moves (and O is rescaled) only when a row max exceeds it by more than TAU.  0 =
+  // rescale exactly when the max changes: with TAU > 0 the largest probability of a
+  // row is no longer exactly 1.0 and its bf16 rounding shows in O.
+  static constexpr float TAU = 0.f;
   static constexpr int BM = 128;
   static constexpr int ELEM = FP8 ? 1 : 2;
   static constexpr int ROW_BYTES = D * ELEM;        // bytes of one tile row
@@ -71,12 +84,12 @@ struct FwdCfg {
   static constexpr int KSTEP_BYTES = MMA_K * ELEM;  // always 32
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_K = Q_BYTES;
-  static constexpr int SMEM_V = SMEM_K + STAGES * KV_BYTES;
-  static constexpr int SMEM_BAR = SMEM_V + STAGES * KV_BYTES;
+  static constexpr int SMEM_V = SMEM_K + KST * KV_BYTES;
+  static constexpr int SMEM_BAR = SMEM_V + VST * KV_BYTES;
   // barriers
   static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_ODONE = 6,
-                       B_DRAIN = 7, B_KFULL = 8, B_VFULL = 8 + STAGES,
-                       B_KVEMPTY = 8 + 2 * STAGES, NBARS = 8 + 3 * STAGES;
+                       B_DRAIN = 7, B_KFULL = 8, B_KEMPTY = 8 + KST, B_VFULL = 8 + 2 * KST,
+                       B_VEMPTY = 8 + 2 * KST + VST, NBARS = 8 + 2 * KST + 2 * VST;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;   // tmem slot, abort flag, reductions
   static constexpr int SMEM_TOTAL = SMEM_MISC + 64;
   static constexpr int SMEM_ALLOC = SMEM_TOTAL + 1024;     // slack to align the base to 1024
@@ -128,8 +141,34 @@ template <class C>
 __device__ void fwd_producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                              const FwdParams& p, uint32_t sbase, uint32_t bars, const WaitCtl& wc) {
   auto bar = [&](int i) { return bars + 8u * i; };
-  uint32_t g = 0, t = 0;
+  // Loads follow the order the MMA warp consumes them: per item Q, K_0, then
+  // (K_j, V_{j-1}) for j >= 1, then V_{n-1}; K therefore runs one step ahead of V.
+  uint32_t gk = 0, gv = 0, t = 0;   // K loads, V loads, items issued so far
   bool ok = true;
+  auto load_k = [&](int j, int bh) -> bool {
+    const int s = gk % C::KST;
+    if (gk >= C::KST && !mbar_wait(bar(C::B_KEMPTY + s), ((gk / C::KST) - 1) & 1, wc, kSiteKVEmpty))
+      return false;
+    mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::KV_BYTES);
+#pragma unroll
+    for (int c = 0; c < C::NBOX; ++c)
+      tma_load_3d(sbase + C::SMEM_K + s * C::KV_BYTES + c * C::BN * 128, tk, bar(C::B_KFULL + s),
+                  c * C::BOX_ELEMS, j * C::BN, bh);
+    ++gk;
+    return true;
+  };
+  auto load_v = [&](int j, int bh) -> bool {
+    const int s = gv % C::VST;
+    if (gv >= C::VST && !mbar_wait(bar(C::B_VEMPTY + s), ((gv / C::VST) - 1) & 1, wc, kSiteKVEmpty))
+      return false;
+    mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::KV_BYTES);
+#pragma unroll
+    for (int c = 0; c < C::NBOX; ++c)
+      tma_load_3d(sbase + C::SMEM_V + s * C::KV_BYTES + c * C::BN * 128, tv, bar(C::B_VFULL + s),
+                  c * C::BOX_ELEMS, j * C::BN, bh);
+    ++gv;
+    return true;
+  };
   for (int k = 0; ok; ++k) {
     const int w = fwd_item_index(k);
     if (w >= p.total_items) break;
@@ -142,41 +181,28 @@ __device__ void fwd_producer(const CUtensorMap* tq, const CUtensorMap* tk, const
     for (int c = 0; c < C::NBOX; ++c)
       tma_load_3d(sbase + C::SMEM_Q + c * C::BM * 128, tq, bar(C::B_QFULL), c * C::BOX_ELEMS,
                   qt * C::BM, bh);
-    for (int j = 0; j < n; ++j) {
-      const uint32_t gj = g + j;
-      const int s = gj % C::STAGES;
-      if (gj >= C::STAGES &&
-          !(ok = mbar_wait(bar(C::B_KVEMPTY + s), ((gj / C::STAGES) - 1) & 1, wc, kSiteKVEmpty)))
-        break;
-      mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::KV_BYTES);
-#pragma unroll
-      for (int c = 0; c < C::NBOX; ++c)
-        tma_load_3d(sbase + C::SMEM_K + s * C::KV_BYTES + c * C::BN * 128, tk,
-                    bar(C::B_KFULL + s), c * C::BOX_ELEMS, j * C::BN, bh);
-      mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::KV_BYTES);
-#pragma unroll
-      for (int c = 0; c < C::NBOX; ++c)
-        tma_load_3d(sbase + C::SMEM_V + s * C::KV_BYTES + c * C::BN * 128, tv,
-                    bar(C::B_VFULL + s), c * C::BOX_ELEMS, j * C::BN, bh);
-    }
-    g += n;
     ++t;
+    if (!(ok = load_k(0, bh))) break;
+    for (int j = 1; j < n && ok; ++j) ok = load_k(j, bh) && load_v(j - 1, bh);
+    if (ok) ok = load_v(n - 1, bh);
   }
   if (!ok) {
     // Aborted: let the tile copies already issued land before the CTA exits.
-    if (t > 0 || g > 0) mbar_wait_drain(bar(C::B_QFULL), (t > 0 ? t - 1 : 0) & 1, 100000000ull);
-    for (uint32_t gk = (g > C::STAGES ? g - C::STAGES : 0); gk < g; ++gk) {
-      mbar_wait_drain(bar(C::B_KFULL + gk % C::STAGES), (gk / C::STAGES) & 1, 100000000ull);
-      mbar_wait_drain(bar(C::B_VFULL + gk % C::STAGES), (gk / C::STAGES) & 1, 100000000ull);
-    }
+    if (t > 0) mbar_wait_drain(bar(C::B_QFULL), (t - 1) & 1, 100000000ull);
+    for (uint32_t i = (gk > C::KST ? gk - C::KST : 0); i < gk; ++i)
+      mbar_wait_drain(bar(C::B_KFULL + i % C::KST), (i / C::KST) & 1, 100000000ull);
+    for (uint32_t i = (gv > C::VST ? gv - C::VST : 0); i < gv; ++i)
+      mbar_wait_drain(bar(C::B_VFULL + i % C::VST), (i / C::VST) & 1, 100000000ull);
     return;
   }
   // Drain: wait until the MMA side has released every buffer, so no tensor-core
   // commit is still due to arrive on this CTA's barriers when it exits.
   if (t > 0) {
     ok = mbar_wait(bar(C::B_QEMPTY), (t - 1) & 1, wc, kSiteQEmpty);
-    for (uint32_t gk = (g > C::STAGES ? g - C::STAGES : 0); ok && gk < g; ++gk)
-      ok = mbar_wait(bar(C::B_KVEMPTY + gk % C::STAGES), (gk / C::STAGES) & 1, wc, kSiteKVEmpty);
+    for (uint32_t i = (gk > C::KST ? gk - C::KST : 0); ok && i < gk; ++i)
+      ok = mbar_wait(bar(C::B_KEMPTY + i % C::KST), (i / C::KST) & 1, wc, kSiteKVEmpty);
+    for (uint32_t i = (gv > C::VST ? gv - C::VST : 0); ok && i < gv; ++i)
+      ok = mbar_wait(bar(C::B_VEMPTY + i % C::VST), (i / C::VST) & 1, wc, kSiteKVEmpty);
   }
 }
 
@@ -196,8 +222,8 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint3
   auto issue_pv = [&](uint32_t gk, bool first) -> bool {
     const int b = gk & 1;
     if (!mbar_wait(bar(C::B_PFULL + b), (gk >> 1) & 1, wc, kSitePFull)) return false;
-    const int s = gk % C::STAGES;
-    if (!mbar_wait(bar(C::B_VFULL + s), (gk / C::STAGES) & 1, wc, kSiteVFull)) return false;
+    const int s = gk % C::VST;
+    if (!mbar_wait(bar(C::B_VFULL + s), (gk / C::VST) & 1, wc, kSiteVFull)) return false;
     tc_fence_after();
     const uint32_t vbase = sbase + C::SMEM_V + s * C::KV_BYTES;
 #pragma unroll
@@ -208,7 +234,7 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint3
       const uint32_t a_tmem = tmem + C::TM_S + b * C::BN + kb * (C::MMA_K * C::ELEM / 4);
       umma_ts<C::FP8>(tmem + C::TM_O, a_tmem, bdesc, IDESC_O, (first && kb == 0) ? 0u : 1u);
     }
-    tc_commit(bar(C::B_KVEMPTY + s));
+    tc_commit(bar(C::B_VEMPTY + s));
     tc_commit(bar(C::B_ODONE));
     return true;
   };
@@ -223,8 +249,8 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint3
     tc_fence_after();
     for (int j = 0; j < n && ok; ++j) {
       const uint32_t gj = g + j;
-      const int s = gj % C::STAGES;
-      if (!(ok = mbar_wait(bar(C::B_KFULL + s), (gj / C::STAGES) & 1, wc, kSiteKFull))) break;
+      const int s = gj % C::KST;
+      if (!(ok = mbar_wait(bar(C::B_KFULL + s), (gj / C::KST) & 1, wc, kSiteKFull))) break;
       tc_fence_after();
       const int b = gj & 1;
       const uint32_t kbase = sbase + C::SMEM_K + s * C::KV_BYTES;
@@ -238,6 +264,7 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint3
         const uint64_t bdesc = sdesc_sw128(kbase + box * C::BN * 128 + off, 16, 1024);
         umma_ss<C::FP8>(tmem + C::TM_S + b * C::BN, adesc, bdesc, IDESC_S, kb > 0 ? 1u : 0u);
       }
+      tc_commit(bar(C::B_KEMPTY + s));
       tc_commit(bar(C::B_SFULL + b));
       if (j == n - 1) tc_commit(bar(C::B_QEMPTY));
       if (j > 0) ok = issue_pv(gj - 1, j == 1);
@@ -250,6 +277,37 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint3
   tc_commit(bar(C::B_DRAIN));
   if (!mbar_wait_drain(bar(C::B_DRAIN), 0, wc.timeout_ns))
     atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
+}
+
+// ---------------------------------------------------------------- software exp2
+// 2^x for a pair of fp32 values on the FMA/ALU pipes instead of the special-function
+// unit (the issoh.co.jp page, section FA4のB200で1613TFLOPs…, on why Blackwell needs
+// part of the exponentials in software).  Cody-Waite reduction x = n + f with
+// n = rint(x) (added to 1.5*2^23 so n lands in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial with minimax relative error 7.5e-5
+// (coefficients from csrc/fit_exp2_poly.py); 2^n by adding n << 23 to the
+// exponent field.  x is clamped at -126 (the result there, about 1.2e-38, stands in
+// for anything smaller), so the exponent field never underflows; valid for x <= 127.
+// Only used on tiles with no masked scores, so a masked -inf never reaches it.
+__device__ __forceinline__ uint64_t ex2_poly_pair(uint64_t x2) {
+  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f,
+                  kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+  float xa, xb;
+  f2_unpack(x2, xa, xb);
+  const uint64_t x = f2_pack(fmaxf(xa, -126.f), fmaxf(xb, -126.f));
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
+  const uint64_t nf = f2_add(t, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(nf, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f2_pack(kC3, kC3), f, f2_pack(kC2, kC2));
+  p = f2_fma(p, f, f2_pack(kC1, kC1));
+  p = f2_fma(p, f, f2_pack(kC0, kC0));
+  float pa, pb, ta, tb;
+  f2_unpack(p, pa, pb);
+  f2_unpack(t, ta, tb);
+  const uint32_t ra = __float_as_uint(pa) + (__float_as_uint(ta) << 23);
+  const uint32_t rb = __float_as_uint(pb) + (__float_as_uint(tb) << 23);
+  return f2_pack(__uint_as_float(ra), __uint_as_float(rb));
 }
 
 // ---------------------------------------------------------------- softmax warps
@@ -290,14 +348,19 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
       const int b = gj & 1;
       if (!(ok = mbar_wait(bar(C::B_SFULL + b), (gj >> 1) & 1, wc, kSiteSFull))) break;
       tc_fence_after();
+      // the whole score row of this thread in one TMEM load
       float s[C::BN];
+      {
+        uint32_t r[C::BN];
+        if constexpr (C::BN == 128) {
+          tmem_ld128(lane_base + C::TM_S + b * C::BN, r);
+          tmem_ld_wait128(r);
+        } else {
+          tmem_ld64(lane_base + C::TM_S + b * C::BN, r);
+          tmem_ld_wait64(r);
+        }
 #pragma unroll
-      for (int c = 0; c < C::BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + C::TM_S + b * C::BN + c, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < C::BN; ++i) s[i] = __uint_as_float(r[i]);
       }
       const int kv0 = j * C::BN;
       const bool need_mask = (p.causal && kv0 + C::BN - 1 > qt * C::BM) || (kv0 + C::BN > p.N);
@@ -313,19 +376,53 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
         c_j = sl2 * qsc * p.k_scale[bh * p.n_st + j];
         fold = 256.f * p.v_scale[bh * p.n_st + j] / vmax;
       }
-      float mx = s[0];
+      // row max: four independent three-input chains
+      float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-      for (int c = 1; c < C::BN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m, mx * c_j);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2(m - m_use);          // 0 on the first tile (m = -inf)
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < C::BN; ++c) {
-        s[c] = ex2(fmaf(s[c], c_j, -m_use));
-        sum += s[c];
+      for (int c = 0; c < C::BN; c += 8) {
+        a0 = max3f(a0, s[c], s[c + 1]);
+        a1 = max3f(a1, s[c + 2], s[c + 3]);
+        a2 = max3f(a2, s[c + 4], s[c + 5]);
+        a3 = max3f(a3, s[c + 6], s[c + 7]);
       }
-      l = l * alpha + sum;
+      const float m_cand = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * c_j;
+      // Reference max: moved only when the row max rises by more than TAU (log2
+      // units); P then stays <= 2^TAU and the final O / l is unchanged.
+      const bool raise = m_cand > m + C::TAU;
+      const float m_new = raise ? m_cand : m;
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = raise ? ex2(m - m_use) : 1.f;   // 0 on the first tile (m = -inf)
+      // P = 2^(S c - m): pairs through the f32x2 FMA; most exponentials on the
+      // special-function unit, EMU of every 4 pairs on the FMA pipe.
+      const uint64_t c2 = f2_pack(c_j, c_j);
+      const uint64_t nm2 = f2_pack(-m_use, -m_use);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      // masked tiles (diagonal / ragged) use the special-function unit throughout, so a
+      // masked score gives exactly 0
+      auto exps = [&](auto emu_tag) {
+        constexpr int kEmu = decltype(emu_tag)::value;
+#pragma unroll
+        for (int c = 0; c < C::BN; c += 2) {
+          const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c2, nm2);
+          uint64_t p2;
+          if ((c / 2) % 4 < kEmu) {
+            p2 = ex2_poly_pair(x2);
+          } else {
+            float xa, xb;
+            f2_unpack(x2, xa, xb);
+            p2 = f2_pack(ex2(xa), ex2(xb));
+          }
+          acc[(c / 2) % 4] = f2_add(acc[(c / 2) % 4], p2);
+          f2_unpack(p2, s[c], s[c + 1]);
+        }
+      };
+      if (need_mask)
+        exps(std::integral_constant<int, 0>{});
+      else
+        exps(std::integral_constant<int, C::EMU>{});
+      float sa, sb;
+      f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
+      l = l * alpha + (sa + sb);
       // P -> tensor memory over the consumed S columns
       if constexpr (C::FP8) {
 #pragma unroll
@@ -351,8 +448,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
       if (j > 0) {
         if (!(ok = mbar_wait(bar(C::B_ODONE), (gj - 1) & 1, wc, kSiteODone))) break;
         tc_fence_after();
-        const bool changed = m_new > m;
-        if (__any_sync(0xffffffffu, changed)) {
+        if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
           for (int c = 0; c < C::D; c += 32) {
             uint32_t r[32];
