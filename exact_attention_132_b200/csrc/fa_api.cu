@@ -14,6 +14,8 @@
 #include "fa.h"
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd_pp.cuh"
+#include "fa_fwd_ws.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa {
@@ -170,20 +172,110 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, FwdParams p, c
   return FA_OK;
 }
 
+// Two query tiles per CTA (fa_fwd_pp.cuh) for d <= 128.
+template <class C>
+fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p,
+                        cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  if (fa_status s = device_info(&di)) return s;
+  CUtensorMap mq, mk, mv;
+  if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
+  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
+  auto kern = fa_fwd_pp_kernel<C>;
+  if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
+  {
+    // The kernel re-splits its registers between warpgroups (setmaxnreg); the split
+    // must fit the launch allocation or the growing warpgroups would wait forever.
+    cudaFuncAttributes fa_attr;
+    cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+    if (fa_attr.numRegs * C::THREADS < 2 * 128 * C::REGS_SOFTMAX + 128 * C::REGS_OTHER)
+      return fail(FA_ERR_CUDA, "forward kernel built with %d registers/thread: too few for its "
+                  "register split", fa_attr.numRegs);
+  }
+  const int tiles = (p.N + C::BM - 1) / C::BM;
+  p.n_qt = (tiles + 1) / 2;                       // query-tile PAIRS per head
+  p.n_kt = (p.N + C::BN - 1) / C::BN;
+  p.n_st = (p.N + 127) / 128;
+  p.total_items = p.BH * p.n_qt;
+  p.group_heads = causal_group_heads(p.BH, 2ll * p.N * C::D * C::ELEM);
+  p.status = di->status;
+  p.timeout_ns = kWaitTimeoutNs;
+  const int grid = p.total_items < di->sms ? p.total_items : di->sms;
+  kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
+  return FA_OK;
+}
+
+// One query tile per CTA, split softmax, two output accumulators (fa_fwd_ws.cuh).
+template <class C>
+fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p,
+                        cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  if (fa_status s = device_info(&di)) return s;
+  CUtensorMap mq, mk, mv;
+  if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
+  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
+  auto kern = fa_fwd_ws_kernel<C>;
+  if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
+  p.n_qt = (p.N + C::BM - 1) / C::BM;
+  p.n_kt = (p.N + C::BN - 1) / C::BN;
+  p.n_st = (p.N + 127) / 128;
+  p.total_items = p.BH * p.n_qt;
+  p.group_heads = causal_group_heads(p.BH, 2ll * p.N * C::D * C::ELEM);
+  p.status = di->status;
+  p.timeout_ns = kWaitTimeoutNs;
+  const int grid = p.total_items < di->sms ? p.total_items : di->sms;
+  kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
+  return FA_OK;
+}
+
 // Tuning knobs (compile-time): software-exp2 share and pipeline depth.
 #ifndef FA_FWD_EMU
 #define FA_FWD_EMU 1
 #endif
+#ifndef FA_FWD_EMU_MQ
+#define FA_FWD_EMU_MQ FA_FWD_EMU
+#endif
 #ifndef FA_FWD_D128_KST
-#define FA_FWD_D128_KST 3
+#define FA_FWD_D128_KST 2
 #endif
 #ifndef FA_FWD_D128_VST
 #define FA_FWD_D128_VST 2
 #endif
+// d <= 128 kernel: 2 = split softmax + two accumulators, 1 = two query tiles, 0 = one tile
+#ifndef FA_FWD_PINGPONG
+#define FA_FWD_PINGPONG 2
+#endif
+#ifndef FA_FWD_TAU
+#define FA_FWD_TAU 0
+#endif
+#ifndef FA_FWD_EXPH
+#define FA_FWD_EXPH 0
+#endif
+#if FA_FWD_PINGPONG == 2
+using FwdD64 = WSCfg<64, 4, 4, false, FA_FWD_EMU, FA_FWD_EMU_MQ>;
+using FwdD128 = WSCfg<128, FA_FWD_D128_KST, FA_FWD_D128_VST, false, FA_FWD_EMU, FA_FWD_EMU_MQ>;
+using FwdF8D128 = WSCfg<128, 4, 4, true, FA_FWD_EMU, FA_FWD_EMU_MQ>;
+#define FA_LAUNCH_FWD_SMALL launch_fwd_ws
+#elif FA_FWD_PINGPONG == 1
+using FwdD64 = PPCfg<64, 4, 4, false, FA_FWD_EMU, FA_FWD_TAU, FA_FWD_EXPH>;
+using FwdD128 = PPCfg<128, FA_FWD_D128_KST, FA_FWD_D128_VST, false, FA_FWD_EMU, FA_FWD_TAU,
+                      FA_FWD_EXPH>;
+using FwdF8D128 = PPCfg<128, 4, 4, true, FA_FWD_EMU>;
+#define FA_LAUNCH_FWD_SMALL launch_fwd_pp
+#else
 using FwdD64 = FwdCfg<64, 128, 4, 4, false, FA_FWD_EMU>;
-using FwdD128 = FwdCfg<128, 128, FA_FWD_D128_KST, FA_FWD_D128_VST, false, FA_FWD_EMU>;
-using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_EMU>;
+using FwdD128 = FwdCfg<128, 128, 3, 2, false, FA_FWD_EMU>;
 using FwdF8D128 = FwdCfg<128, 128, 4, 4, true, FA_FWD_EMU>;
+#define FA_LAUNCH_FWD_SMALL launch_fwd
+#endif
+using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_EMU>;
 
 using DkdvD64 = DkdvCfg<64, 64, 128, 3>;
 using DkdvD128 = DkdvCfg<128, 128, 128, 2>;
@@ -326,8 +418,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.lse = lse;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 64: return launch_fwd<FwdD64>(q, k, v, p, st);
-    case 128: return launch_fwd<FwdD128>(q, k, v, p, st);
+    case 64: return FA_LAUNCH_FWD_SMALL<FwdD64>(q, k, v, p, st);
+    case 128: return FA_LAUNCH_FWD_SMALL<FwdD128>(q, k, v, p, st);
     default: return launch_fwd<FwdD256>(q, k, v, p, st);
   }
 }
@@ -357,7 +449,7 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
-  return launch_fwd<FwdF8D128>(q8, k8, v8, p, static_cast<cudaStream_t>(stream));
+  return FA_LAUNCH_FWD_SMALL<FwdF8D128>(q8, k8, v8, p, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {

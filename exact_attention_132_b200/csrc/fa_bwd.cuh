@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i)
-      mbar_init(bar(i), (i == C::B_P || i == C::B_DS) ? 128u : 1u);
+      mbar_init(bar(i), (i == C::B_P || i == C::B_DS) ? 4u : 1u);   // 4 compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_P));
+      mbar_arrive_warp(bar(C::B_P));
       // dS^T row = P^T * (dP^T - D_q), written as bf16 over the consumed dP^T columns
 #pragma unroll
       for (int c0 = 0; c0 < C::BMQ; c0 += 32) {
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_DS));
+      mbar_arrive_warp(bar(C::B_DS));
     }
     // epilogue: dV and scale*dK -> bf16 global
     if (ok && mbar_wait(bar(C::B_ACC), 0, wc, kSiteDqDone)) {
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int nsteps = p.causal ? min(p.n_kt, ((qt + 1) * C::BM - 1) / C::BN + 1) : p.n_kt;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NBARS; ++i) mbar_init(bar(i), i == C::B_DS ? 128u : 1u);
+    for (int i = 0; i < C::NBARS; ++i) mbar_init(bar(i), i == C::B_DS ? 4u : 1u);   // 4 warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_DS));
+      mbar_arrive_warp(bar(C::B_DS));
     }
     if (ok && mbar_wait(bar(C::B_ACC), 0, wc, kSiteDqDone)) {
       tc_fence_after();

@@ -310,6 +310,24 @@ __device__ __forceinline__ uint64_t ex2_poly_pair(uint64_t x2) {
   return f2_pack(__uint_as_float(ra), __uint_as_float(rb));
 }
 
+// 2^x for a pair of fp32 values on the special-function unit in half precision:
+// one ex2.approx.f16x2 for both.  The argument is rounded to f16 (relative 2^-11,
+// so an absolute error below 0.004 for |x| <= 8); results below the f16 range
+// become 0.  Returned as fp32.
+__device__ __forceinline__ uint64_t ex2_f16_pair(uint64_t x2) {
+  float xa, xb;
+  f2_unpack(x2, xa, xb);
+  uint32_t h, e;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(xb), "f"(xa));
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
+  float ra, rb;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
+      : "=f"(ra), "=f"(rb)
+      : "r"(e));
+  return f2_pack(ra, rb);
+}
+
 // ---------------------------------------------------------------- softmax warps
 template <class C>
 __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, const WaitCtl& wc) {
@@ -463,7 +481,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
       m = m_new;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_PFULL + b));
+      mbar_arrive_warp(bar(C::B_PFULL + b));
     }
     if (!ok) break;
     // epilogue: O / l -> bf16 -> global; row logsumexp
@@ -512,7 +530,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i) {
       uint32_t cnt = 1;
-      if (i == C::B_PFULL || i == C::B_PFULL + 1) cnt = 128;
+      if (i == C::B_PFULL || i == C::B_PFULL + 1) cnt = 4;   // one arrival per softmax warp
       mbar_init(bars + 8u * i, cnt);
     }
     *abort_flag = 0;

@@ -18,7 +18,7 @@ constexpr unsigned kStatusTimeout = 4u << 24;
 
 enum WaitSite : unsigned {
   kSiteQFull = 1, kSiteQEmpty, kSiteKFull, kSiteVFull, kSiteKVEmpty, kSiteSFull, kSitePFull,
-  kSiteODone, kSiteDrain, kSiteDsFull, kSiteDqDone, kSiteSelfTest = 99
+  kSiteODone, kSiteDrain, kSiteDsFull, kSiteDqDone, kSiteXchg, kSiteSelfTest = 99
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -56,6 +56,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_try_wait, but the thread may stay suspended (issuing nothing) for up to
+// `hint_ns` while the phase is incomplete; it resumes when the phase completes.  Keeps
+// a waiting thread from taking issue slots from the other warps on its SM sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// One arrival per warp instead of one per thread (a barrier takes its arrivals one at
+// a time, so 32 per warp cost hundreds of cycles).  The warp barrier orders every
+// lane's earlier writes -- shared-memory stores, or tensor-memory stores completed by
+// tcgen05.wait::st and fenced by tcgen05.fence::before_thread_sync -- before lane 0's
+// release-arrive.  Barrier counts are in warps.
+__device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
 
 // Shared control block of one CTA: abort flag plus where to report.
 struct WaitCtl {
@@ -64,13 +88,15 @@ struct WaitCtl {
   uint64_t timeout_ns;        // bound of every wait
 };
 
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& c,
+// Inlined on purpose: a shared out-of-line callee cannot serve warps whose register
+// budgets differ after setmaxnreg.
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& c,
                                             unsigned site) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*c.abort_flag) return false;
     if (global_timer_ns() - t0 > c.timeout_ns) {
       atomicCAS(c.status, 0u, kStatusTimeout | site);
@@ -92,7 +118,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 
 // Wait used only while shutting down after an abort: ignores the abort flag so
 // that in-flight copies and MMAs are waited for, still bounded by `timeout_ns`.
-__device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (global_timer_ns() - t0 > timeout_ns) return false;
@@ -214,6 +240,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
       FA_S8(0), FA_S8(8)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {"
+      "%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
+      FA_S8(0), FA_S8(8), FA_S8(16), FA_S8(24), FA_S8(32), FA_S8(40), FA_S8(48), FA_S8(56)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st128(uint32_t taddr, const uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x128.b32 [%0], {"
+      "%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127,%128};" ::"r"(taddr),
+      FA_S8(0), FA_S8(8), FA_S8(16), FA_S8(24), FA_S8(32), FA_S8(40), FA_S8(48), FA_S8(56), FA_S8(64), FA_S8(72), FA_S8(80), FA_S8(88), FA_S8(96), FA_S8(104), FA_S8(112), FA_S8(120)
       : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() {
@@ -338,6 +378,77 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
+}
+
+// Re-split the block's registers between warpgroups (every warp of a warpgroup must
+// execute the same instruction).  The shares must add up to at most the block's
+// launch allocation (threads x registers per thread at launch), or an .inc waits.
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ----------------------------------------------------------------------------- warp-uniform issue
+// The issuing warps run their loops with all 32 lanes (warp-uniform control flow, so
+// descriptors and addresses stay in uniform registers) and let exactly one lane, chosen
+// by elect.sync, issue each MMA, commit or TMA copy.
+__device__ __forceinline__ void umma_ss_elect(bool fp8, uint32_t d_tmem, uint64_t adesc,
+                                              uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  if (fp8)
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_ts_elect(bool fp8, uint32_t d_tmem, uint32_t a_tmem,
+                                              uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  if (fp8)
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+          bar)
+      : "memory");
+}
+__device__ __forceinline__ bool elect_one() {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 x;\n\telect.sync x|e, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, e;\n\t}\n"
+      : "=r"(r));
+  return r != 0;
+}
+// Bounded wait by a whole warp; every lane returns the same answer.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtl& c,
+                                               unsigned site) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, c, site));
 }
 
 // Named barrier among `nthreads` threads (ids 1..15; 0 is __syncthreads).
