@@ -41,21 +41,24 @@ HEADLINE = "fwd_d128"
 METRIC = "attention TFLOP/s fwd and fwd+bwd on 1 B200; % of dense BF16/FP8 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per launch of the forward kernel at the headline workload,
-# from ncu's dram__bytes_read.sum + dram__bytes_write.sum (profiles/
-# fa_fwd_d128_causal_B4H16N4096.md), keyed by the hash of the kernel sources they were
-# measured on.  A changed kernel has no entry and reports traffic = null.
-FWD_TRAFFIC_BYTES = {"785b081eb6926ca8": 279_987_456}
+# DRAM bytes (read + write) per launch of the headline forward kernel, from ncu's
+# dram__bytes_read.sum + dram__bytes_write.sum (profiles/
+# fa_fwd_d128_causal_B4H16N4096.md), keyed by a hash of the kernel sources and the
+# launched kernel's name (which carries its tile configuration).  A changed kernel has
+# no entry and reports traffic = null.
+FWD_TRAFFIC_BYTES = {"cbd65f6503dfa87d": 267_930_880}
 KERNEL_SOURCES = ("exact_attention_132_b200/csrc/fa_fwd.cuh",
+                  "exact_attention_132_b200/csrc/fa_fwd_ws.cuh",
                   "exact_attention_132_b200/csrc/sm100_ptx.cuh")
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel_name: str) -> str:
     import hashlib
     parts = []
     for rel in KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             parts.append(hashlib.sha256(f.read()).hexdigest() + "\n")
+    parts.append(kernel_name)
     return hashlib.sha256("".join(parts).encode()).hexdigest()[:16]
 
 
@@ -218,6 +221,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
+    kname = fa.fa_fwd_kernel_name(w.d)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -239,10 +243,10 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_src} bf16 dense matmul (burst)",
-                     "kernel": "fa_fwd_kernel<FwdCfg<128,128,2,false>>",
+                     "kernel": kname,
                      "kernel_ms": round(kernel_ms, 4),
-                     "traffic": FWD_TRAFFIC_BYTES.get(kernel_source_hash()),
-                     "kernel_source_hash": kernel_source_hash()},
+                     "traffic": FWD_TRAFFIC_BYTES.get(kernel_source_hash(kname)),
+                     "kernel_source_hash": kernel_source_hash(kname)},
         "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "ms_per_step": round(e2e_ms / e2e_steps, 4)},

@@ -17,7 +17,8 @@ import torch
 
 __all__ = [
     "FAError", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_size", "fa_last_error_string",
-    "fa_get_device_status", "fa_debug_wait_timeout_selftest", "fa_version", "attention_forward",
+    "fa_get_device_status", "fa_debug_wait_timeout_selftest", "fa_version", "fa_fwd_kernel_name",
+    "attention_forward",
     "attention_forward_fp8", "attention_backward", "LIB_PATH", "lib",
 ]
 
@@ -52,6 +53,8 @@ def _load() -> ctypes.CDLL:
     L.fa_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     L.fa_debug_wait_timeout_selftest.argtypes = [i, vp]
     L.fa_version.argtypes = []
+    L.fa_fwd_kernel_name.argtypes = [i, i]
+    L.fa_fwd_kernel_name.restype = ctypes.c_char_p
     for name in ("fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_get_device_status",
                  "fa_debug_wait_timeout_selftest", "fa_version"):
         getattr(L, name).restype = ctypes.c_int
@@ -184,6 +187,12 @@ def fa_debug_wait_timeout_selftest(timeout_us: int, stream=None) -> None:
 
 def fa_version() -> int:
     return int(lib.fa_version())
+
+
+def fa_fwd_kernel_name(head_dim: int, fp8: bool = False) -> str | None:
+    """Name and tile configuration of the forward kernel launched for this head dim."""
+    r = lib.fa_fwd_kernel_name(int(head_dim), int(bool(fp8)))
+    return None if r is None else r.decode()
 
 
 # ------------------------------------------------------------------ allocating helpers

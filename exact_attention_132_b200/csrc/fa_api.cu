@@ -10,12 +10,14 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include "fa.h"
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd_pp.cuh"
 #include "fa_fwd_ws.cuh"
+#include "fa_fwd_sp.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa {
@@ -219,7 +221,12 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
   if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
   if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
   if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
-  auto kern = fa_fwd_ws_kernel<C>;
+  auto kern = [] {
+    if constexpr (C::SEPARATE_P)
+      return fa_fwd_sp_kernel<C>;
+    else
+      return fa_fwd_ws_kernel<C>;
+  }();
   if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
   p.n_qt = (p.N + C::BM - 1) / C::BM;
   p.n_kt = (p.N + C::BN - 1) / C::BN;
@@ -235,12 +242,18 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
   return FA_OK;
 }
 
-// Tuning knobs (compile-time): software-exp2 share and pipeline depth.
+// Tuning knobs (compile-time): software-exp2 share, pipeline depth, kernel family.
 #ifndef FA_FWD_EMU
 #define FA_FWD_EMU 1
 #endif
 #ifndef FA_FWD_EMU_MQ
 #define FA_FWD_EMU_MQ FA_FWD_EMU
+#endif
+#ifndef FA_FWD_WS_INDEP
+#define FA_FWD_WS_INDEP 1
+#endif
+#ifndef FA_FWD_WS_SPLIT
+#define FA_FWD_WS_SPLIT 0
 #endif
 #ifndef FA_FWD_D128_KST
 #define FA_FWD_D128_KST 2
@@ -248,33 +261,63 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #ifndef FA_FWD_D128_VST
 #define FA_FWD_D128_VST 2
 #endif
-// d <= 128 kernel: 2 = split softmax + two accumulators, 1 = two query tiles, 0 = one tile
-#ifndef FA_FWD_PINGPONG
-#define FA_FWD_PINGPONG 2
-#endif
 #ifndef FA_FWD_TAU
 #define FA_FWD_TAU 0
 #endif
 #ifndef FA_FWD_EXPH
 #define FA_FWD_EXPH 0
 #endif
-#if FA_FWD_PINGPONG == 2
-using FwdD64 = WSCfg<64, 4, 4, false, FA_FWD_EMU, FA_FWD_EMU_MQ>;
-using FwdD128 = WSCfg<128, FA_FWD_D128_KST, FA_FWD_D128_VST, false, FA_FWD_EMU, FA_FWD_EMU_MQ>;
-using FwdF8D128 = WSCfg<128, 4, 4, true, FA_FWD_EMU, FA_FWD_EMU_MQ>;
-#define FA_LAUNCH_FWD_SMALL launch_fwd_ws
-#elif FA_FWD_PINGPONG == 1
-using FwdD64 = PPCfg<64, 4, 4, false, FA_FWD_EMU, FA_FWD_TAU, FA_FWD_EXPH>;
-using FwdD128 = PPCfg<128, FA_FWD_D128_KST, FA_FWD_D128_VST, false, FA_FWD_EMU, FA_FWD_TAU,
-                      FA_FWD_EXPH>;
-using FwdF8D128 = PPCfg<128, 4, 4, true, FA_FWD_EMU>;
-#define FA_LAUNCH_FWD_SMALL launch_fwd_pp
-#else
-using FwdD64 = FwdCfg<64, 128, 4, 4, false, FA_FWD_EMU>;
-using FwdD128 = FwdCfg<128, 128, 3, 2, false, FA_FWD_EMU>;
-using FwdF8D128 = FwdCfg<128, 128, 4, 4, true, FA_FWD_EMU>;
-#define FA_LAUNCH_FWD_SMALL launch_fwd
+// Kernel family per problem class (measured fastest on the causal N = 4096 workloads):
+// 0 = one query tile per CTA (fa_fwd.cuh), 1 = two query tiles (fa_fwd_pp.cuh),
+// 2 = split softmax (fa_fwd_ws.cuh), 3 = separate P buffers (fa_fwd_sp.cuh).
+#ifndef FA_FWD_D64_KIND
+#define FA_FWD_D64_KIND 1
 #endif
+#ifndef FA_FWD_D128_KIND
+#define FA_FWD_D128_KIND 2
+#endif
+#ifndef FA_FWD_F8_KIND
+#define FA_FWD_F8_KIND 1
+#endif
+
+template <int KIND, int D, bool FP8>
+struct FwdPick {
+  // stage depths: deep rings where shared memory allows, 2 + 2 for bf16 d = 128
+  static constexpr bool kWide = (D == 128 && !FP8);
+  static constexpr int KST = kWide ? FA_FWD_D128_KST : 4;
+  static constexpr int VST = kWide ? FA_FWD_D128_VST : 4;
+  using Cfg = std::conditional_t<
+      KIND == 0, FwdCfg<D, 128, kWide ? 3 : 4, kWide ? 2 : 4, FP8, FA_FWD_EMU>,
+      std::conditional_t<
+          KIND == 1, PPCfg<D, KST, VST, FP8, FA_FWD_EMU, FA_FWD_TAU, FA_FWD_EXPH>,
+          std::conditional_t<KIND == 2,
+                             WSCfg<D, KST, VST, FP8, FA_FWD_EMU, FA_FWD_EMU_MQ,
+                                   FA_FWD_WS_SPLIT != 0, FA_FWD_WS_INDEP != 0>,
+                             SPCfg<D, KST, VST, FP8, FA_FWD_EMU>>>>;
+  static const char* name() {
+    static const std::string n = [] {
+      static const char* fam[] = {"fa_fwd_kernel<FwdCfg", "fa_fwd_pp_kernel<PPCfg",
+                                  "fa_fwd_ws_kernel<WSCfg", "fa_fwd_sp_kernel<SPCfg"};
+      char buf[128];
+      std::snprintf(buf, sizeof buf, "%s<%d,KST%d,VST%d,%s>>", fam[KIND], D, Cfg::KST, Cfg::VST,
+                    FP8 ? "e4m3" : "bf16");
+      return std::string(buf);
+    }();
+    return n.c_str();
+  }
+  static fa_status launch(const void* q, const void* k, const void* v, FwdParams p,
+                          cudaStream_t st) {
+    if constexpr (KIND == 0)
+      return launch_fwd<Cfg>(q, k, v, p, st);
+    else if constexpr (KIND == 1)
+      return launch_fwd_pp<Cfg>(q, k, v, p, st);
+    else
+      return launch_fwd_ws<Cfg>(q, k, v, p, st);
+  }
+};
+using FwdD64 = FwdPick<FA_FWD_D64_KIND, 64, false>;
+using FwdD128 = FwdPick<FA_FWD_D128_KIND, 128, false>;
+using FwdF8D128 = FwdPick<FA_FWD_F8_KIND, 128, true>;
 using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_EMU>;
 
 using DkdvD64 = DkdvCfg<64, 64, 128, 3>;
@@ -418,8 +461,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.lse = lse;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 64: return FA_LAUNCH_FWD_SMALL<FwdD64>(q, k, v, p, st);
-    case 128: return FA_LAUNCH_FWD_SMALL<FwdD128>(q, k, v, p, st);
+    case 64: return FwdD64::launch(q, k, v, p, st);
+    case 128: return FwdD128::launch(q, k, v, p, st);
     default: return launch_fwd<FwdD256>(q, k, v, p, st);
   }
 }
@@ -449,7 +492,7 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
-  return FA_LAUNCH_FWD_SMALL<FwdF8D128>(q8, k8, v8, p, static_cast<cudaStream_t>(stream));
+  return FwdF8D128::launch(q8, k8, v8, p, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -562,5 +605,20 @@ fa_status fa_debug_wait_timeout_selftest(int timeout_us, void* stream) {
 }
 
 int fa_version(void) { return 100; }
+
+const char* fa_fwd_kernel_name(int head_dim, int fp8) {
+  using namespace fa;
+  if (fp8) return head_dim == 128 ? FwdF8D128::name() : nullptr;
+  switch (head_dim) {
+    case 64: return FwdD64::name();
+    case 128: return FwdD128::name();
+    case 256: {
+      static const std::string n = "fa_fwd_kernel<FwdCfg<256,KST" + std::to_string(FwdD256::KST) +
+                                   ",VST" + std::to_string(FwdD256::VST) + ",bf16>>";
+      return n.c_str();
+    }
+    default: return nullptr;
+  }
+}
 
 }  // extern "C"

@@ -27,7 +27,8 @@
 
 namespace fa {
 
-template <int D_, int KST_, int VST_, bool FP8_, int EMU_ = 1, int EMU_MQ_ = EMU_>
+template <int D_, int KST_, int VST_, bool FP8_, int EMU_ = 1, int EMU_MQ_ = EMU_, bool SPLIT_ = false,
+          bool INDEP_ = false>
 struct WSCfg {
   static constexpr int D = D_;
   static constexpr int BN = 128;
@@ -36,6 +37,15 @@ struct WSCfg {
   static constexpr bool FP8 = FP8_;
   static constexpr int EMU = EMU_;
   static constexpr int EMU_MQ = EMU_MQ_;             // same, for the MMA warp's quadrant
+  // Issue S = Q K^T and O += P V from two warps on different SM sub-partitions: a
+  // sub-partition's instruction queue holds each tcgen05.mma until the tensor core
+  // takes it, so one issuing warp delays the softmax warps beside it.
+  static constexpr bool SPLIT = SPLIT_;
+  // Independent row halves: each half-warp keeps its own running max and sum and its
+  // own output accumulator O_h (h = column half of the scores), so the two halves of a
+  // row never wait for each other inside the key loop; they are combined once per tile.
+  static constexpr bool INDEP = INDEP_;
+  static constexpr bool SEPARATE_P = false;
   static constexpr int HALF = BN / 2;                 // score columns per softmax warp
   static constexpr int DH = D / 2;                    // output columns per softmax warp
   static constexpr int ELEM = FP8 ? 1 : 2;
@@ -57,15 +67,19 @@ struct WSCfg {
   static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_ODONE = 6,
                        B_DRAIN = 7, B_XCHG = 8, B_KFULL = 12, B_KEMPTY = 12 + KST,
                        B_VFULL = 12 + 2 * KST, B_VEMPTY = 12 + 2 * KST + VST,
-                       NBARS = 12 + 2 * KST + 2 * VST;
+                       B_PVDONE = 12 + 2 * KST + 2 * VST, B_DRAIN2 = B_PVDONE + 2,
+                       B_PFULLH = B_DRAIN2 + 1,          // + 2 * half + buffer, 4 warps each
+                       B_PVDONEH = B_PFULLH + 4,         // + half
+                       NBARS = B_PVDONEH + 2;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
   static constexpr int TM_S = 0;                      // + b * BN
   static constexpr int TM_O = 2 * BN;                 // + a * D
   static constexpr int TM_COLS = 512;
   static constexpr int THREADS = 384;
-  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, PV_WARP = 10;
   static_assert(2 * BN + 2 * D <= TM_COLS, "tensor memory budget");
+  static_assert(!(SPLIT && INDEP), "one issuer layout at a time");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(DH % 32 == 0, "32-column output chunks per warp");
 };
@@ -227,6 +241,87 @@ __device__ void ws_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32
   }
   tc_commit_elect(bars + 8u * C::B_DRAIN);
   if (!mbar_wait_drain(bars + 8u * C::B_DRAIN, 0, wc.timeout_ns) && (threadIdx.x & 31) == 0)
+    atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
+}
+
+// ---------------------------------------------------------------- split issuers
+// S issuer (the TMEM owner's warp).  S(j) reuses the buffer of S(j-2), whose P the
+// product P(j-2) V reads: S(j) is issued only once that product is complete, which
+// also keeps "S(j) complete => P(j-2) V complete" true for the softmax warps.
+template <class C>
+__device__ void ws_mma_s(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                         const WaitCtl& wc) {
+  const uint32_t b_qfull = bars + 8u * C::B_QFULL, b_qempty = bars + 8u * C::B_QEMPTY;
+  const uint32_t b_sfull = bars + 8u * C::B_SFULL, b_pvdone = bars + 8u * C::B_PVDONE;
+  const uint32_t b_kfull = bars + 8u * C::B_KFULL, b_kempty = bars + 8u * C::B_KEMPTY;
+  const uint64_t qdesc = sdesc_sw128(sbase + C::SMEM_Q, 16, 1024);
+  const uint64_t kdesc_base = sdesc_sw128(sbase + C::SMEM_K, 16, 1024);
+  uint32_t g = 0, t = 0;
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int w = fwd_item_index(k);
+    if (w >= p.total_items) break;
+    int bh, qt;
+    fwd_decode_item(p, w, bh, qt);
+    const int n = fwd_num_kv_tiles<C>(p, qt);
+    if (!mbar_wait_warp(b_qfull, t & 1, wc, kSiteQFull)) { ok = false; break; }
+    for (int j = 0; j < n; ++j) {
+      const uint32_t gj = g + j;
+      const uint32_t ks = gj % C::KST;
+      if (!mbar_wait_warp(b_kfull + 8u * ks, (gj / C::KST) & 1, wc, kSiteKFull)) { ok = false; break; }
+      if (gj >= 2 && !mbar_wait_warp(b_pvdone + 8u * (gj & 1), ((gj - 2) >> 1) & 1, wc, kSitePFull)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      ws_issue_s<C>(tmem + C::TM_S + (gj & 1) * C::BN, qdesc,
+                    kdesc_base + static_cast<uint64_t>(ks * (C::KV_BYTES >> 4)));
+      tc_commit_elect(b_kempty + 8u * ks);
+      tc_commit_elect(b_sfull + 8u * (gj & 1));
+      if (j == n - 1) tc_commit_elect(b_qempty);
+    }
+    if (!ok) break;
+    g += n;
+    ++t;
+  }
+  tc_commit_elect(bars + 8u * C::B_DRAIN);
+  if (!mbar_wait_drain(bars + 8u * C::B_DRAIN, 0, wc.timeout_ns) && (threadIdx.x & 31) == 0)
+    atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
+}
+
+// P V issuer: P(j) V into O_{j%2}; each accumulator is overwritten on its first use.
+template <class C>
+__device__ void ws_mma_pv(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                          const WaitCtl& wc) {
+  const uint32_t b_pfull = bars + 8u * C::B_PFULL, b_pvdone = bars + 8u * C::B_PVDONE;
+  const uint32_t b_odone = bars + 8u * C::B_ODONE;
+  const uint32_t b_vfull = bars + 8u * C::B_VFULL, b_vempty = bars + 8u * C::B_VEMPTY;
+  const uint64_t vdesc_base = sdesc_sw128(sbase + C::SMEM_V, C::BN * 128, 1024);
+  uint32_t g = 0;
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int w = fwd_item_index(k);
+    if (w >= p.total_items) break;
+    int bh, qt;
+    fwd_decode_item(p, w, bh, qt);
+    const int n = fwd_num_kv_tiles<C>(p, qt);
+    for (int j = 0; j < n; ++j) {
+      const uint32_t gp = g + j;
+      const uint32_t vs = gp % C::VST;
+      if (!mbar_wait_warp(b_pfull + 8u * (gp & 1), (gp >> 1) & 1, wc, kSitePFull)) { ok = false; break; }
+      if (!mbar_wait_warp(b_vfull + 8u * vs, (gp / C::VST) & 1, wc, kSiteVFull)) { ok = false; break; }
+      tc_fence_after();
+      ws_issue_pv<C>(tmem + C::TM_O + (j & 1) * C::D, tmem + C::TM_S + (gp & 1) * C::BN,
+                     vdesc_base + static_cast<uint64_t>(vs * (C::KV_BYTES >> 4)), j < 2);
+      tc_commit_elect(b_vempty + 8u * vs);
+      tc_commit_elect(b_pvdone + 8u * (gp & 1));
+      if (j == n - 1) tc_commit_elect(b_odone);
+    }
+    if (!ok) break;
+    g += n;
+  }
+  tc_commit_elect(bars + 8u * C::B_DRAIN2);
+  if (!mbar_wait_drain(bars + 8u * C::B_DRAIN2, 0, wc.timeout_ns) && (threadIdx.x & 31) == 0)
     atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
 }
 
@@ -446,6 +541,302 @@ __device__ void ws_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, flo
   }
 }
 
+// ---------------------------------------------------------------- independent halves
+// P_h(j) V_h into O_h, h = 0, 1: the key block of half h is keys [64h, 64h + 64) of the
+// tile; its probabilities sit at columns [64h, 64h + P_COLS_H) of the S buffer, inside
+// the columns that half's own scores occupied.
+template <class C>
+__device__ __forceinline__ void ws_issue_pv_half(uint32_t o_tmem, uint32_t s_tmem, uint64_t vdesc,
+                                                 int h, bool first) {
+  constexpr uint32_t IDESC_O = C::FP8 ? idesc_e4m3(128, C::D, true) : idesc_bf16(128, C::D, true);
+  constexpr int KB_H = C::HALF / C::MMA_K;                  // MMAs per half
+#pragma unroll
+  for (int i = 0; i < KB_H; ++i) {
+    const int kb = h * KB_H + i;
+    umma_ts_elect(C::FP8, o_tmem, s_tmem + h * C::HALF + i * (C::MMA_K * C::ELEM / 4),
+                  vdesc + static_cast<uint64_t>((kb * C::MMA_K * 128) >> 4), IDESC_O,
+                  (first && i == 0) ? 0u : 1u);
+  }
+}
+
+template <class C>
+__device__ void ws_mma_indep(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                             const WaitCtl& wc) {
+  const uint32_t b_qfull = bars + 8u * C::B_QFULL, b_qempty = bars + 8u * C::B_QEMPTY;
+  const uint32_t b_sfull = bars + 8u * C::B_SFULL, b_pfullh = bars + 8u * C::B_PFULLH;
+  const uint32_t b_pvdoneh = bars + 8u * C::B_PVDONEH, b_odone = bars + 8u * C::B_ODONE;
+  const uint32_t b_kfull = bars + 8u * C::B_KFULL, b_kempty = bars + 8u * C::B_KEMPTY;
+  const uint32_t b_vfull = bars + 8u * C::B_VFULL, b_vempty = bars + 8u * C::B_VEMPTY;
+  const uint64_t qdesc = sdesc_sw128(sbase + C::SMEM_Q, 16, 1024);
+  const uint64_t kdesc_base = sdesc_sw128(sbase + C::SMEM_K, 16, 1024);
+  const uint64_t vdesc_base = sdesc_sw128(sbase + C::SMEM_V, C::BN * 128, 1024);
+  uint32_t g = 0, t = 0;
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int w = fwd_item_index(k);
+    if (w >= p.total_items) break;
+    int bh, qt;
+    fwd_decode_item(p, w, bh, qt);
+    const int n = fwd_num_kv_tiles<C>(p, qt);
+    if (!mbar_wait_warp(b_qfull, t & 1, wc, kSiteQFull)) { ok = false; break; }
+    tc_fence_after();
+    for (int j = 0; j <= n; ++j) {
+      const uint32_t gj = g + j;
+      if (j < n) {
+        // S(j) into S_{gj%2}: the P V products that read the buffer's last P were
+        // issued earlier by this thread and complete first
+        const uint32_t ks = gj % C::KST;
+        if (!mbar_wait_warp(b_kfull + 8u * ks, (gj / C::KST) & 1, wc, kSiteKFull)) { ok = false; break; }
+        tc_fence_after();
+        ws_issue_s<C>(tmem + C::TM_S + (gj & 1) * C::BN, qdesc,
+                      kdesc_base + static_cast<uint64_t>(ks * (C::KV_BYTES >> 4)));
+        tc_commit_elect(b_kempty + 8u * ks);
+        tc_commit_elect(b_sfull + 8u * (gj & 1));
+        if (j == n - 1) tc_commit_elect(b_qempty);
+      }
+      if (j > 0) {
+        const uint32_t gp = gj - 1;
+        const uint32_t vs = gp % C::VST;
+        const uint32_t pb = gp & 1, pph = (gp >> 1) & 1;
+        if (!mbar_wait_warp(b_vfull + 8u * vs, (gp / C::VST) & 1, wc, kSiteVFull)) { ok = false; break; }
+        const uint64_t vdesc = vdesc_base + static_cast<uint64_t>(vs * (C::KV_BYTES >> 4));
+        const uint32_t s_tmem = tmem + C::TM_S + pb * C::BN;
+        if (j == 1) {
+          // first products of a tile overwrite both accumulators: wait until both
+          // halves are past the previous tile's epilogue, which reads both
+          if (!mbar_wait_warp(b_pfullh + 8u * pb, pph, wc, kSitePFull) ||
+              !mbar_wait_warp(b_pfullh + 8u * (2 + pb), pph, wc, kSitePFull)) {
+            ok = false;
+            break;
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (j > 1 && !mbar_wait_warp(b_pfullh + 8u * (2 * h + pb), pph, wc, kSitePFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          ws_issue_pv_half<C>(tmem + C::TM_O + h * C::D, s_tmem, vdesc, h, j == 1);
+          tc_commit_elect(b_pvdoneh + 8u * h);
+        }
+        if (!ok) break;
+        tc_commit_elect(b_vempty + 8u * vs);
+        if (j == n) tc_commit_elect(b_odone);
+      }
+    }
+    if (!ok) break;
+    g += n;
+    ++t;
+  }
+  tc_commit_elect(bars + 8u * C::B_DRAIN);
+  if (!mbar_wait_drain(bars + 8u * C::B_DRAIN, 0, wc.timeout_ns) && (threadIdx.x & 31) == 0)
+    atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
+}
+
+// Scale a full output accumulator row (D columns) of this warp's lanes by `a`, in
+// 32-column pieces.
+template <class C>
+__device__ __forceinline__ void ws_scale_o_full(uint32_t taddr, float a) {
+  const uint64_t a2 = f2_pack(a, a);
+#pragma unroll 1
+  for (int c = 0; c < C::D; c += 64) {
+    uint32_t r[64];
+    tmem_ld64(taddr + c, r);
+    tmem_ld_wait64(r);
+#pragma unroll
+    for (int i = 0; i < 64; i += 2) {
+      float x, y;
+      f2_unpack(f2_mul(f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), a2), x, y);
+      r[i] = __float_as_uint(x);
+      r[i + 1] = __float_as_uint(y);
+    }
+    tmem_st64(taddr + c, r);
+  }
+}
+
+template <class C>
+__device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tmem, float* xbuf,
+                                 const WaitCtl& wc) {
+  const int warp = threadIdx.x / 32;
+  const int quad = warp & 3, half = warp >> 2;
+  const int row = quad * 32 + (threadIdx.x & 31);
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+  const uint32_t b_sfull = bars + 8u * C::B_SFULL;
+  const uint32_t b_pfull = bars + 8u * (C::B_PFULLH + 2 * half);
+  const uint32_t b_pvdone = bars + 8u * (C::B_PVDONEH + half);
+  const uint32_t b_odone = bars + 8u * C::B_ODONE;
+  const uint32_t b_x = bars + 8u * (C::B_XCHG + quad);
+  const uint32_t o_mine = lane_base + C::TM_O + half * C::D;
+  uint32_t xc = 0;
+  const float LOG2E = 1.4426950408889634f;
+  const float LN2 = 0.6931471805599453f;
+  const float sl2 = p.scale * LOG2E;
+  __nv_bfloat16* o_out = reinterpret_cast<__nv_bfloat16*>(p.o);
+  uint32_t g = 0, t = 0;
+  bool ok = true;
+
+  for (int k = 0; ok; ++k) {
+    const int w = fwd_item_index(k);
+    if (w >= p.total_items) break;
+    int bh, qt;
+    fwd_decode_item(p, w, bh, qt);
+    const int n = fwd_num_kv_tiles<C>(p, qt);
+    const int q_idx = qt * C::BM + row;
+    float m = -INFINITY, l = 0.f;
+    float qsc = 1.f, vmax = 1.f;
+    if constexpr (C::FP8) {
+      qsc = p.q_scale[bh * p.n_st + qt];
+      vmax = 0.f;
+      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[bh * p.n_st + j]);
+    }
+    for (int j = 0; j < n; ++j) {
+      const uint32_t gj = g + j;
+      const uint32_t b = gj & 1;
+      if (!mbar_wait(b_sfull + 8u * b, (gj >> 1) & 1, wc, kSiteSFull)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t s_cols = lane_base + C::TM_S + b * C::BN + half * C::HALF;
+      float s[C::HALF];
+      {
+        uint32_t r[C::HALF];
+        tmem_ld64(s_cols, r);
+        tmem_ld_wait64(r);
+#pragma unroll
+        for (int i = 0; i < C::HALF; ++i) s[i] = __uint_as_float(r[i]);
+      }
+      const int kv0 = j * C::BN + half * C::HALF;
+      // warp-uniform: some row of this warp has a key of this half beyond its limit
+      const bool need_mask = (p.causal && kv0 + C::HALF - 1 > qt * C::BM + quad * 32) ||
+                             (kv0 + C::HALF > p.N);
+      if (need_mask) {
+        const int lim = p.causal ? min(q_idx, p.N - 1) : p.N - 1;
+#pragma unroll
+        for (int c = 0; c < C::HALF; ++c)
+          if (kv0 + c > lim) s[c] = -INFINITY;
+      }
+      float c_j = sl2, fold = 1.f;
+      if constexpr (C::FP8) {
+        c_j = sl2 * qsc * p.k_scale[bh * p.n_st + j];
+        fold = 256.f * p.v_scale[bh * p.n_st + j] / vmax;
+      }
+      float mx[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(s[2 * i], s[2 * i + 1]);
+#pragma unroll
+      for (int c = 8; c < C::HALF; c += 8)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = max3f(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
+      const float m_cand = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c_j;
+      const bool raise = m_cand > m;
+      const float m_new = raise ? m_cand : m;
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = raise ? ex2(m - m_use) : 1.f;
+      const uint64_t c2 = f2_pack(c_j, c_j);
+      const uint64_t nm2 = f2_pack(-m_use, -m_use);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      auto exps = [&](auto emu_tag) {
+        constexpr int kEmu = decltype(emu_tag)::value;
+#pragma unroll
+        for (int c = 0; c < C::HALF; c += 2) {
+          const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c2, nm2);
+          uint64_t p2;
+          if ((c / 2) % 4 < kEmu) {
+            p2 = ex2_poly_pair(x2);
+          } else {
+            float xa, xb;
+            f2_unpack(x2, xa, xb);
+            p2 = f2_pack(ex2(xa), ex2(xb));
+          }
+          acc[(c / 2) % 4] = f2_add(acc[(c / 2) % 4], p2);
+          f2_unpack(p2, s[c], s[c + 1]);
+        }
+      };
+      if (need_mask)
+        exps(std::integral_constant<int, 0>{});
+      else if (quad == (C::MMA_WARP & 3))
+        exps(std::integral_constant<int, C::EMU_MQ>{});
+      else
+        exps(std::integral_constant<int, C::EMU>{});
+      float sa, sb;
+      f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
+      l = l * alpha + (sa + sb);
+      // P_h(j) over this half's own score columns
+      if constexpr (C::FP8) {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          r[i] = pack_e4m3x4(s[4 * i] * fold, s[4 * i + 1] * fold, s[4 * i + 2] * fold,
+                             s[4 * i + 3] * fold);
+        tmem_st16(s_cols, r);
+      } else {
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
+        tmem_st32(s_cols, r);
+      }
+      // O_h was last updated by P_h(j-1) V_h: once it is complete, scale it to the
+      // new reference max (warp-uniform decision; alpha = 1 on rows that kept theirs)
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+        if (!mbar_wait(b_pvdone, (gj - 1) & 1, wc, kSitePvDone)) { ok = false; break; }
+        tc_fence_after();
+        ws_scale_o_full<C>(o_mine, alpha);
+      }
+      m = m_new;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive_warp(b_pfull + 8u * b);
+    }
+    if (!ok) break;
+    if (!mbar_wait(b_odone, t & 1, wc, kSiteODone)) { ok = false; break; }
+    ++t;
+    tc_fence_after();
+    // combine the halves: O = sum_h O_h 2^(m_h - m), l = sum_h l_h 2^(m_h - m)
+    xbuf[half * 128 + row] = m;
+    xbuf[(2 + half) * 128 + row] = l;
+    mbar_arrive_warp(b_x);
+    if (!mbar_wait(b_x, xc & 1, wc, kSiteXchg)) { ok = false; break; }
+    ++xc;
+    const float m_o = xbuf[(half ^ 1) * 128 + row];
+    const float l_o = xbuf[(2 + (half ^ 1)) * 128 + row];
+    const float m_fin = fmaxf(m, m_o);
+    const float m_ref = (m_fin == -INFINITY) ? 0.f : m_fin;
+    const float e_me = ex2(((m == -INFINITY) ? m_ref : m) - m_ref) * (m == -INFINITY ? 0.f : 1.f);
+    const float e_ot = ex2(((m_o == -INFINITY) ? m_ref : m_o) - m_ref) * (m_o == -INFINITY ? 0.f : 1.f);
+    const float l_row = l * e_me + l_o * e_ot;
+    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / l_row;
+    const float w_self = e_me * inv_l, w_other = e_ot * inv_l;
+    const float w0 = half == 0 ? w_self : w_other;
+    const float w1 = half == 0 ? w_other : w_self;
+    const bool row_ok = q_idx < p.N;
+    __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * C::D + half * C::DH;
+#pragma unroll 1
+    for (int c = 0; c < C::DH; c += 32) {
+      uint32_t a0[32], a1[32];
+      tmem_ld32(lane_base + C::TM_O + half * C::DH + c, a0);
+      tmem_ld32(lane_base + C::TM_O + C::D + half * C::DH + c, a1);
+      tmem_ld_wait(a0);
+      tmem_ld_wait(a1);
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float x0 = fmaf(__uint_as_float(a1[2 * i]), w1, __uint_as_float(a0[2 * i]) * w0);
+        const float y0 = fmaf(__uint_as_float(a1[2 * i + 1]), w1, __uint_as_float(a0[2 * i + 1]) * w0);
+        pk[i] = pack_bf16x2(x0, y0);
+      }
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      }
+    }
+    if (half == 0 && row_ok && p.lse != nullptr)
+      p.lse[static_cast<size_t>(bh) * p.N + q_idx] = (m_ref + __log2f(l_row)) * LN2;
+    tc_fence_before();
+    g += n;
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     fa_fwd_ws_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -464,6 +855,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int i = 0; i < C::NBARS; ++i) {
       uint32_t cnt = 1;
       if (i == C::B_PFULL || i == C::B_PFULL + 1) cnt = 8;           // the 8 softmax warps
+      if (i >= C::B_PFULLH && i < C::B_PFULLH + 4) cnt = 4;           // one column half
       if (i >= C::B_XCHG && i < C::B_XCHG + 4) cnt = 2;               // one half-warp pair
       mbar_init(bars + 8u * i, cnt);
     }
@@ -486,9 +878,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (warp == C::PRODUCER_WARP) {
     ws_producer<C>(&tq, &tk, &tv, p, sbase, bars, wc);
   } else if (warp == C::MMA_WARP) {
-    ws_mma<C>(p, sbase, bars, tmem, wc);
+    if constexpr (C::SPLIT)
+      ws_mma_s<C>(p, sbase, bars, tmem, wc);
+    else if constexpr (C::INDEP)
+      ws_mma_indep<C>(p, sbase, bars, tmem, wc);
+    else
+      ws_mma<C>(p, sbase, bars, tmem, wc);
+  } else if (C::SPLIT && warp == C::PV_WARP) {
+    ws_mma_pv<C>(p, sbase, bars, tmem, wc);
   } else if (warp < 8) {
-    ws_softmax<C>(p, bars, tmem, xbuf, wc);
+    if constexpr (C::INDEP)
+      ws_softmax_indep<C>(p, bars, tmem, xbuf, wc);
+    else
+      ws_softmax<C>(p, bars, tmem, xbuf, wc);
   }
 
   tc_fence_before();

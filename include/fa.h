@@ -170,6 +170,15 @@ fa_status fa_debug_wait_timeout_selftest(int timeout_us, void* stream);
 /* fa_version — library version, major*10000 + minor*100 + patch. */
 int fa_version(void);
 
+/*
+ * fa_fwd_kernel_name — name of the forward kernel that fa_fwd (fp8 = 0) or
+ * fa_fwd_fp8 (fp8 != 0) launches for head dimension `head_dim`, with its
+ * tile configuration, e.g. "fa_fwd_ws_kernel<WSCfg<128,KST2,VST2,bf16>>".  The
+ * string is static and owned by the library.  Returns NULL for an unsupported
+ * head dimension.  Host only; launches nothing.
+ */
+const char* fa_fwd_kernel_name(int head_dim, int fp8);
+
 #ifdef __cplusplus
 }
 #endif

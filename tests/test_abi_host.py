@@ -39,6 +39,16 @@ def test_version():
     assert fa.fa_version() >= 100
 
 
+def test_forward_kernel_names():
+    # every supported head dim names a kernel whose tile matches it; others name none
+    for d, fp8 in ((64, False), (128, False), (256, False), (128, True)):
+        name = fa.fa_fwd_kernel_name(d, fp8)
+        assert name and name.startswith("fa_fwd_") and f"<{d}," in name
+        assert ("e4m3" in name) == fp8
+    assert fa.fa_fwd_kernel_name(96) is None
+    assert fa.fa_fwd_kernel_name(64, True) is None
+
+
 def _fwd(q=1, k=1, v=1, o=1, lse=None, B=1, H=1, N=128, d=128, scale=0.1, causal=0):
     P = lambda x: None if x is None else ctypes.c_void_p(16 * x)
     return fa.lib.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, scale, causal, None)
