@@ -255,6 +255,9 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #ifndef FA_FWD_WS_SPLIT
 #define FA_FWD_WS_SPLIT 0
 #endif
+#ifndef FA_FWD_SP_SPLIT
+#define FA_FWD_SP_SPLIT 1
+#endif
 #ifndef FA_FWD_D128_KST
 #define FA_FWD_D128_KST 2
 #endif
@@ -293,7 +296,7 @@ struct FwdPick {
           std::conditional_t<KIND == 2,
                              WSCfg<D, KST, VST, FP8, FA_FWD_EMU, FA_FWD_EMU_MQ,
                                    FA_FWD_WS_SPLIT != 0, FA_FWD_WS_INDEP != 0>,
-                             SPCfg<D, KST, VST, FP8, FA_FWD_EMU>>>>;
+                             SPCfg<D, KST, VST, FP8, FA_FWD_EMU, FA_FWD_SP_SPLIT != 0>>>>;
   static const char* name() {
     static const std::string n = [] {
       static const char* fam[] = {"fa_fwd_kernel<FwdCfg", "fa_fwd_pp_kernel<PPCfg",

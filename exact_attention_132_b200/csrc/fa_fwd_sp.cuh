@@ -20,7 +20,8 @@
 //    issued a whole softmax step earlier, so the wait is normally already satisfied.
 //
 // Roles: warps 0-7 softmax (warp w: lanes 32*(w%4).., column half w/4), warp 8 TMA
-// producer, warp 9 MMA issuer + TMEM owner, warps 10-11 idle (warpgroup alignment).
+// producer, warp 9 S issuer + TMEM owner, warp 10 P V issuer (warp 9 issues both when
+// SPLIT is off), warp 11 idle (warpgroup alignment).
 // Tensor memory: S [0,128), P_0 [128,192), P_1 [192,256), O_0 [256,256+D), O_1 [256+D,256+2D).
 #pragma once
 
@@ -30,7 +31,7 @@
 
 namespace fa {
 
-template <int D_, int KST_, int VST_, bool FP8_, int EMU_ = 1>
+template <int D_, int KST_, int VST_, bool FP8_, int EMU_ = 1, bool SPLIT_ = true>
 struct SPCfg {
   static constexpr int D = D_;
   static constexpr int BN = 128;
@@ -39,6 +40,10 @@ struct SPCfg {
   static constexpr bool FP8 = FP8_;
   static constexpr int EMU = EMU_;                    // software exp2 share, in quarters
   static constexpr bool SEPARATE_P = true;
+  // Two issuing warps: S = Q K^T from one, the P V products from another.  The two
+  // streams share no tensor-memory buffer, so neither waits for the other, and each
+  // warp's barrier waits overlap the other's MMAs.
+  static constexpr bool SPLIT = SPLIT_;
   static constexpr int HALF = BN / 2;                 // score columns per softmax warp
   static constexpr int DH = D / 2;                    // output columns written per warp
   static constexpr int ELEM = FP8 ? 1 : 2;
@@ -59,11 +64,12 @@ struct SPCfg {
   static constexpr int SMEM_BAR = SMEM_X + 4 * 128 * 4;
   static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_SEMPTY = 3, B_ODONE = 4,
                        B_DRAIN = 5,
-                       B_XCHG = 6,                    // + quad, one arrival per half-warp
-                       B_PFULLH = 10,                 // + 2 * half + buffer, 4 warps each
-                       B_PVDONEH = 14,                // + half
-                       B_KFULL = 16, B_KEMPTY = 16 + KST, B_VFULL = 16 + 2 * KST,
-                       B_VEMPTY = 16 + 2 * KST + VST, NBARS = 16 + 2 * KST + 2 * VST;
+                       B_DRAIN2 = 6,                  // drain of the P V issuer
+                       B_XCHG = 7,                    // + quad, one arrival per half-warp
+                       B_PFULLH = 11,                 // + 2 * half + buffer, 4 warps each
+                       B_PVDONEH = 15,                // + half
+                       B_KFULL = 17, B_KEMPTY = 17 + KST, B_VFULL = 17 + 2 * KST,
+                       B_VEMPTY = 17 + 2 * KST + VST, NBARS = 17 + 2 * KST + 2 * VST;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
   static constexpr int TM_S = 0;
@@ -71,7 +77,7 @@ struct SPCfg {
   static constexpr int TM_O = 2 * BN;                 // + half * D
   static constexpr int TM_COLS = 512;
   static constexpr int THREADS = 384;
-  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, PV_WARP = 10;
   static_assert(TM_O + 2 * D <= TM_COLS, "tensor memory budget");
   static_assert(2 * PCOL_H <= 64, "P buffer width");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -165,6 +171,99 @@ __device__ void sp_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32
   }
   tc_commit_elect(bars + 8u * C::B_DRAIN);
   if (!mbar_wait_drain(bars + 8u * C::B_DRAIN, 0, wc.timeout_ns) && (threadIdx.x & 31) == 0)
+    atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
+}
+
+// ---------------------------------------------------------------- split issuers
+// S issuer (warp MMA_WARP, also the TMEM owner).
+template <class C>
+__device__ void sp_mma_s(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                         const WaitCtl& wc) {
+  const uint32_t b_qfull = bars + 8u * C::B_QFULL, b_qempty = bars + 8u * C::B_QEMPTY;
+  const uint32_t b_sfull = bars + 8u * C::B_SFULL, b_sempty = bars + 8u * C::B_SEMPTY;
+  const uint32_t b_kfull = bars + 8u * C::B_KFULL, b_kempty = bars + 8u * C::B_KEMPTY;
+  const uint64_t qdesc = sdesc_sw128(sbase + C::SMEM_Q, 16, 1024);
+  const uint64_t kdesc_base = sdesc_sw128(sbase + C::SMEM_K, 16, 1024);
+  uint32_t g = 0, t = 0;
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int w = fwd_item_index(k);
+    if (w >= p.total_items) break;
+    int bh, qt;
+    fwd_decode_item(p, w, bh, qt);
+    const int n = fwd_num_kv_tiles<C>(p, qt);
+    if (!mbar_wait_warp(b_qfull, t & 1, wc, kSiteQFull)) { ok = false; break; }
+    for (int j = 0; j < n; ++j) {
+      const uint32_t gj = g + j;
+      const uint32_t ks = gj % C::KST;
+      if (!mbar_wait_warp(b_kfull + 8u * ks, (gj / C::KST) & 1, wc, kSiteKFull)) { ok = false; break; }
+      if (gj > 0 && !mbar_wait_warp(b_sempty, (gj - 1) & 1, wc, kSiteSFull)) { ok = false; break; }
+      tc_fence_after();
+      ws_issue_s<C>(tmem + C::TM_S, qdesc, kdesc_base + static_cast<uint64_t>(ks * (C::KV_BYTES >> 4)));
+      tc_commit_elect(b_kempty + 8u * ks);
+      tc_commit_elect(b_sfull);
+      if (j == n - 1) tc_commit_elect(b_qempty);
+    }
+    if (!ok) break;
+    g += n;
+    ++t;
+  }
+  tc_commit_elect(bars + 8u * C::B_DRAIN);
+  if (!mbar_wait_drain(bars + 8u * C::B_DRAIN, 0, wc.timeout_ns) && (threadIdx.x & 31) == 0)
+    atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
+}
+
+// P V issuer (warp PV_WARP): P_h(j) V_h into O_h as each half's probabilities arrive.
+template <class C>
+__device__ void sp_mma_pv(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                          const WaitCtl& wc) {
+  const uint32_t b_pfullh = bars + 8u * C::B_PFULLH, b_pvdoneh = bars + 8u * C::B_PVDONEH;
+  const uint32_t b_odone = bars + 8u * C::B_ODONE;
+  const uint32_t b_vfull = bars + 8u * C::B_VFULL, b_vempty = bars + 8u * C::B_VEMPTY;
+  const uint64_t vdesc_base = sdesc_sw128(sbase + C::SMEM_V, C::BN * 128, 1024);
+  uint32_t g = 0;
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int w = fwd_item_index(k);
+    if (w >= p.total_items) break;
+    int bh, qt;
+    fwd_decode_item(p, w, bh, qt);
+    const int n = fwd_num_kv_tiles<C>(p, qt);
+    for (int j = 0; j < n; ++j) {
+      const uint32_t gp = g + j;
+      const uint32_t vs = gp % C::VST;
+      const uint32_t pb = gp & 1, pph = (gp >> 1) & 1;
+      if (!mbar_wait_warp(b_vfull + 8u * vs, (gp / C::VST) & 1, wc, kSiteVFull)) { ok = false; break; }
+      const uint64_t vdesc = vdesc_base + static_cast<uint64_t>(vs * (C::KV_BYTES >> 4));
+      if (j == 0) {
+        // the first products of a tile overwrite both accumulators: both halves must
+        // be past the previous tile's epilogue, which reads both
+        if (!mbar_wait_warp(b_pfullh + 8u * pb, pph, wc, kSitePFull) ||
+            !mbar_wait_warp(b_pfullh + 8u * (2 + pb), pph, wc, kSitePFull)) {
+          ok = false;
+          break;
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (j > 0 && !mbar_wait_warp(b_pfullh + 8u * (2 * h + pb), pph, wc, kSitePFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        sp_issue_pv_half<C>(tmem + C::TM_O + h * C::D, tmem + C::TM_P + pb * 64 + h * C::PCOL_H,
+                            vdesc, h, j == 0);
+        tc_commit_elect(b_pvdoneh + 8u * h);
+      }
+      if (!ok) break;
+      tc_commit_elect(b_vempty + 8u * vs);
+      if (j == n - 1) tc_commit_elect(b_odone);
+    }
+    if (!ok) break;
+    g += n;
+  }
+  tc_commit_elect(bars + 8u * C::B_DRAIN2);
+  if (!mbar_wait_drain(bars + 8u * C::B_DRAIN2, 0, wc.timeout_ns) && (threadIdx.x & 31) == 0)
     atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
 }
 
@@ -414,7 +513,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (warp == C::PRODUCER_WARP) {
     ws_producer<C>(&tq, &tk, &tv, p, sbase, bars, wc);
   } else if (warp == C::MMA_WARP) {
-    sp_mma<C>(p, sbase, bars, tmem, wc);
+    if constexpr (C::SPLIT)
+      sp_mma_s<C>(p, sbase, bars, tmem, wc);
+    else
+      sp_mma<C>(p, sbase, bars, tmem, wc);
+  } else if (C::SPLIT && warp == C::PV_WARP) {
+    sp_mma_pv<C>(p, sbase, bars, tmem, wc);
   } else if (warp < 8) {
     sp_softmax<C>(p, bars, tmem, xbuf, wc);
   }
