@@ -14,15 +14,16 @@
 //   1. fa_bwd_rowdot   D_i = dO_i . O_i into the caller's workspace (HBM-bound).
 //   2. fa_bwd_dkdv     one CTA per (head, 128-row key tile[, half of d]); it keeps
 //                      K, V in shared memory and dK, dV accumulators in tensor
-//                      memory, and streams the query tiles.  Thread t of the
-//                      compute warps owns key row t (transposed tiles S^T, dP^T).
+//                      memory, and streams the query tiles.  Lane t of the compute
+//                      warps owns key row t (transposed tiles S^T, dP^T).
 //   3. fa_bwd_dq       one CTA per (head, 128-row query tile); it keeps Q, dO in
 //                      shared memory and dQ in tensor memory, and streams K/V.
 // Splitting dQ into its own pass costs a second recompute of S and dP but needs
 // no fp32 atomics and is deterministic.
 //
-// Roles in kernels 2 and 3: warp 0 = TMA producer, warp 1 = MMA issuer (one
-// thread, owns tensor memory), warps 2..5 = elementwise work on TMEM lanes.
+// Roles in kernels 2 and 3: warps 0..7 elementwise work (two warps per TMEM lane
+// quadrant, each on half of the streamed tile's columns), warp 8 TMA producer, warp 9
+// MMA issuer (one elected lane issues; owns tensor memory).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -75,7 +76,20 @@ __global__ void __launch_bounds__(256) fa_bwd_rowdot(const __nv_bfloat16* __rest
 }
 
 // --------------------------------------------------------------------------- 2. dK, dV
-template <int D_, int DH_, int BMQ_, int STAGES_>
+// One CTA per (head, 128-row key tile[, part of d]).  K and V stay in shared memory,
+// dV and dK accumulate in tensor memory, and the query tiles stream through a ring.
+// Per query tile i (BMQ rows):
+//   S^T = K Q_i^T, dP^T = V dO_i^T                      (tensor core, into TMEM)
+//   P^T = 2^(S^T scale log2e - lse_i log2e)           (compute warps, bf16 over S^T)
+//   dV += P^T dO_i                                      (tensor core, A = P^T from TMEM)
+//   dS^T = P^T (dP^T - D_i)                             (compute warps, bf16 over dP^T)
+//   dK += dS^T Q_i                                      (tensor core, A = dS^T from TMEM)
+// S^T and dP^T have SB / DB buffers, so the products of tile i+1 run on the tensor
+// core while the compute warps work on tile i.  Eight compute warps: two per TMEM lane
+// quadrant, each owning half of the BMQ query columns (P needs no row reduction, so
+// the halves never talk to each other).  Each half writes its bf16 P^T / dS^T into
+// the first half of its own column range.
+template <int D_, int DH_, int BMQ_, int STAGES_, int SB_, int DB_, int EMU_ = 1>
 struct DkdvCfg {
   static constexpr int D = D_;          // head dim (contraction of S^T and dP^T)
   static constexpr int DH = DH_;        // columns of dK/dV this CTA produces
@@ -83,6 +97,9 @@ struct DkdvCfg {
   static constexpr int BMQ = BMQ_;      // query rows per streamed tile
   static constexpr int BN = 128;        // key rows of the CTA = TMEM lanes
   static constexpr int STAGES = STAGES_;
+  static constexpr int SB = SB_, DB = DB_;
+  static constexpr int EMU = EMU_;      // software exp2 share, in quarters
+  static constexpr int CH = BMQ / 2;    // query columns per compute warp
   static constexpr int ROW_BYTES = D * 2;
   static constexpr int NBOX = ROW_BYTES / 128;
   static constexpr int KT_BYTES = BN * ROW_BYTES;       // K or V tile
@@ -94,22 +111,70 @@ struct DkdvCfg {
   static constexpr int SMEM_LSE = SMEM_DO + STAGES * QT_BYTES;    // [STAGES][BMQ] fp32
   static constexpr int SMEM_DD = SMEM_LSE + STAGES * BMQ * 4;     // [STAGES][BMQ] fp32
   static constexpr int SMEM_BAR = SMEM_DD + STAGES * BMQ * 4;
-  static constexpr int B_KV = 0, B_SDP = 1, B_P = 2, B_DS = 3, B_ACC = 4, B_DRAIN = 5,
-                       B_FULL = 6, B_EMPTY = 6 + STAGES, NBARS = 6 + 2 * STAGES;
+  static constexpr int B_KV = 0, B_ACC = 1, B_DRAIN = 2,
+                       B_SFULL = 3, B_P = 3 + SB,                   // + buffer
+                       B_DPFULL = 3 + 2 * SB, B_DS = 3 + 2 * SB + DB,
+                       B_FULL = 3 + 2 * SB + 2 * DB, B_EMPTY = B_FULL + STAGES,
+                       NBARS = B_EMPTY + STAGES;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
-  static constexpr int TM_ST = 0, TM_DPT = BMQ, TM_DV = 2 * BMQ, TM_DK = 2 * BMQ + DH;
+  static constexpr int TM_ST = 0;                        // + b * BMQ
+  static constexpr int TM_DPT = SB * BMQ;                // + b * BMQ
+  static constexpr int TM_DV = (SB + DB) * BMQ, TM_DK = TM_DV + DH;
   static constexpr int TM_COLS = 512;
-  static constexpr int THREADS = 192;
-  static_assert(2 * BMQ + 2 * DH <= TM_COLS, "tensor memory budget");
+  static constexpr int THREADS = 320;                    // 8 compute warps, producer, MMA
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+  static_assert((SB + DB) * BMQ + 2 * DH <= TM_COLS, "tensor memory budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-  static_assert(BMQ % 64 == 0 && DH % 64 == 0, "64-column boxes and 32-column TMEM chunks");
+  static_assert(BMQ % 64 == 0 && DH % 64 == 0 && CH % 32 == 0, "box and TMEM chunk sizes");
+  static_assert(SB >= 1 && SB <= 2 && DB >= 1 && DB <= 2, "one or two buffers");
 };
 
 template <class C>
 __device__ __forceinline__ void dkdv_q_range(const BwdParams& p, int kt, int& i0, int& i1) {
   i1 = p.n_qt;
   i0 = p.causal ? (kt * C::BN) / C::BMQ : 0;   // first query tile that reaches key kt*128
+}
+
+// A = (BMQ x 128)^T operand kb (16 query columns) of the bf16 tile written over a
+// BMQ-column fp32 buffer: half h of the columns keeps its values in its own range.
+template <int BMQ>
+__device__ __forceinline__ uint32_t half_packed_col(int kb) {
+  constexpr int KB_H = BMQ / 2 / 16;      // 16-column blocks per half
+  return (kb / KB_H) * (BMQ / 2) + (kb % KB_H) * 8;
+}
+
+// 2^x of an even-length row segment into `pr`: EMU of every 4 pairs on the FMA pipe,
+// the rest on the special-function unit.  x = s * c - b, with b per element (a query
+// column's lse) or one value for the whole segment (the row's lse).
+__device__ __forceinline__ void exp2_pair_into(uint64_t x2, bool soft, float& a, float& b) {
+  if (soft) {
+    f2_unpack(ex2_poly_pair(x2), a, b);
+  } else {
+    float xa, xb;
+    f2_unpack(x2, xa, xb);
+    a = ex2(xa);
+    b = ex2(xb);
+  }
+}
+template <int N, int EMU>
+__device__ __forceinline__ void exp2_row(const uint32_t (&r)[N], float c, const float* b, float (&pr)[N]) {
+  const uint64_t c2 = f2_pack(c, c);
+#pragma unroll
+  for (int i = 0; i < N; i += 2) {
+    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), c2,
+                               f2_pack(-b[i], -b[i + 1]));
+    exp2_pair_into(x2, (i / 2) % 4 < EMU, pr[i], pr[i + 1]);
+  }
+}
+template <int N, int EMU>
+__device__ __forceinline__ void exp2_row(const uint32_t (&r)[N], float c, float b, float (&pr)[N]) {
+  const uint64_t c2 = f2_pack(c, c), nb2 = f2_pack(-b, -b);
+#pragma unroll
+  for (int i = 0; i < N; i += 2) {
+    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), c2, nb2);
+    exp2_pair_into(x2, (i / 2) % 4 < EMU, pr[i], pr[i + 1]);
+  }
 }
 
 template <class C>
@@ -125,11 +190,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   auto bar = [&](int i) { return bars + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
-  float* lse_s = reinterpret_cast<float*>(smem + C::SMEM_LSE);
+  float* lse_s = reinterpret_cast<float*>(smem + C::SMEM_LSE);   // lse * log2(e)
   float* dd_s = reinterpret_cast<float*>(smem + C::SMEM_DD);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const float LOG2E = 1.4426950408889634f;
 
-  // block -> (bh, key tile, d half); heaviest causal tiles (small kt) first
+  // block -> (bh, key tile, d part); heaviest causal tiles (small kt) first
   const int split = blockIdx.x % C::NSPLIT;
   const int rest = blockIdx.x / C::NSPLIT;
   const int kt = rest % p.n_kt;
@@ -139,12 +205,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int nsteps = i1 - i0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NBARS; ++i)
-      mbar_init(bar(i), (i == C::B_P || i == C::B_DS) ? 4u : 1u);   // 4 compute warps
+    for (int i = 0; i < C::NBARS; ++i) {
+      const bool warps8 = (i >= C::B_P && i < C::B_P + C::SB) || (i >= C::B_DS && i < C::B_DS + C::DB);
+      mbar_init(bar(i), warps8 ? 8u : 1u);                  // 8 compute warps arrive
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(tmem_slot), C::TM_COLS);
     tmem_relinquish();
   }
@@ -154,33 +222,31 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == 0) {
-    // ---------------- producer (whole warp: lanes stage lse/D, lane 0 issues TMA)
+  if (warp == C::PRODUCER_WARP) {
+    // ---------------- producer (whole warp: lanes stage lse/D, one lane issues TMA)
     bool ok = true;
-    if (lane == 0) {
+    if (elect_one()) {
       mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KT_BYTES);
       for (int c = 0; c < C::NBOX; ++c) {
         tma_load_3d(sbase + C::SMEM_K + c * C::BN * 128, &tk, bar(C::B_KV), c * 64, kt * C::BN, bh);
         tma_load_3d(sbase + C::SMEM_V + c * C::BN * 128, &tv, bar(C::B_KV), c * 64, kt * C::BN, bh);
       }
     }
+    __syncwarp();
     for (int st = 0; st < nsteps && ok; ++st) {
       const int s = st % C::STAGES;
       const int qi = i0 + st;
-      if (st >= C::STAGES) {
-        // every lane waits; the warp then agrees on the outcome so it stays converged
-        ok = mbar_wait(bar(C::B_EMPTY + s), ((st / C::STAGES) - 1) & 1, wc, kSiteKVEmpty);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-      }
+      if (st >= C::STAGES &&
+          !(ok = mbar_wait_warp(bar(C::B_EMPTY + s), ((st / C::STAGES) - 1) & 1, wc, kSiteKVEmpty)))
+        break;
       for (int c = lane; c < C::BMQ; c += 32) {
         const int q = qi * C::BMQ + c;
         const bool in = q < p.N;
-        lse_s[s * C::BMQ + c] = in ? p.lse[static_cast<size_t>(bh) * p.N + q] : 0.f;
+        lse_s[s * C::BMQ + c] = in ? p.lse[static_cast<size_t>(bh) * p.N + q] * LOG2E : 0.f;
         dd_s[s * C::BMQ + c] = in ? p.drow[static_cast<size_t>(bh) * p.N + q] : 0.f;
       }
       __syncwarp();
-      if (lane == 0) {
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar(C::B_FULL + s), 2 * C::QT_BYTES);
         for (int c = 0; c < C::NBOX; ++c) {
           tma_load_3d(sbase + C::SMEM_Q + s * C::QT_BYTES + c * C::BMQ * 128, &tq,
@@ -189,142 +255,192 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       bar(C::B_FULL + s), c * 64, qi * C::BMQ, bh);
         }
       }
+      __syncwarp();
     }
-    if (lane == 0) {
-      if (ok) {
-        for (int st = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); ok && st < nsteps; ++st)
-          ok = mbar_wait(bar(C::B_EMPTY + st % C::STAGES), (st / C::STAGES) & 1, wc, kSiteKVEmpty);
-      } else {
-        mbar_wait_drain(bar(C::B_KV), 0, 100000000ull);
-        for (int st = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); st < nsteps; ++st)
-          mbar_wait_drain(bar(C::B_FULL + st % C::STAGES), (st / C::STAGES) & 1, 100000000ull);
+    if (ok) {
+      for (int st = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); ok && st < nsteps; ++st)
+        ok = mbar_wait_warp(bar(C::B_EMPTY + st % C::STAGES), (st / C::STAGES) & 1, wc, kSiteKVEmpty);
+    } else {
+      mbar_wait_drain(bar(C::B_KV), 0, 100000000ull);
+      for (int st = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); st < nsteps; ++st)
+        mbar_wait_drain(bar(C::B_FULL + st % C::STAGES), (st / C::STAGES) & 1, 100000000ull);
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ---------------- MMA issuer (whole warp, one elected lane issues)
+    constexpr uint32_t ID_T = idesc_bf16(128, C::BMQ, false);    // S^T, dP^T: 128 x BMQ
+    constexpr uint32_t ID_G = idesc_bf16(128, C::DH, true);      // dV, dK: 128 x DH, B MN-major
+    const int hbox = split * (C::DH / 64);
+    auto qbuf = [&](int st) { return sbase + C::SMEM_Q + (st % C::STAGES) * C::QT_BYTES; };
+    auto dobuf = [&](int st) { return sbase + C::SMEM_DO + (st % C::STAGES) * C::QT_BYTES; };
+    // S^T(st) = K Q^T and, with it or later, dP^T(st) = V dO^T
+    auto issue_st = [&](int st) -> bool {
+      if (!mbar_wait_warp(bar(C::B_FULL + st % C::STAGES), (st / C::STAGES) & 1, wc, kSiteQFull))
+        return false;
+      tc_fence_after();
+#pragma unroll
+      for (int kb = 0; kb < C::D / 16; ++kb) {
+        const int box = kb / 4, off = (kb % 4) * 32;
+        umma_ss_elect(false, tmem + C::TM_ST + (st % C::SB) * C::BMQ,
+                      sdesc_sw128(sbase + C::SMEM_K + box * C::BN * 128 + off, 16, 1024),
+                      sdesc_sw128(qbuf(st) + box * C::BMQ * 128 + off, 16, 1024), ID_T, kb > 0);
+      }
+      tc_commit_elect(bar(C::B_SFULL + st % C::SB));
+      return true;
+    };
+    auto issue_dpt = [&](int st) {
+#pragma unroll
+      for (int kb = 0; kb < C::D / 16; ++kb) {
+        const int box = kb / 4, off = (kb % 4) * 32;
+        umma_ss_elect(false, tmem + C::TM_DPT + (st % C::DB) * C::BMQ,
+                      sdesc_sw128(sbase + C::SMEM_V + box * C::BN * 128 + off, 16, 1024),
+                      sdesc_sw128(dobuf(st) + box * C::BMQ * 128 + off, 16, 1024), ID_T, kb > 0);
+      }
+      tc_commit_elect(bar(C::B_DPFULL + st % C::DB));
+    };
+    bool ok = mbar_wait_warp(bar(C::B_KV), 0, wc, kSiteKFull);
+    // prologue: tile 0's products, then tile 1's where the buffers allow
+    if (ok && nsteps > 0) {
+      ok = issue_st(0);
+      if (ok) issue_dpt(0);
+    }
+    // Tile st+1's products go ahead of tile st's gradient products when they have a
+    // buffer of their own and their query tile can already be resident (a second ring
+    // stage); otherwise they follow them.
+    constexpr bool EARLY_S = C::SB == 2 && C::STAGES >= 2;
+    constexpr bool EARLY_DP = EARLY_S && C::DB == 2;
+    for (int st = 0; st < nsteps && ok; ++st) {
+      const int nx = st + 1;
+      // S^T(st+1) into the other buffer (its last reader, dV(st+1-SB), is issued)
+      if (EARLY_S && nx < nsteps && !(ok = issue_st(nx))) break;
+      if (EARLY_DP && nx < nsteps) issue_dpt(nx);
+      // dV += P^T dO[:, part]   (A = P^T bf16 in TMEM over the S^T columns)
+      if (!(ok = mbar_wait_warp(bar(C::B_P + st % C::SB), (st / C::SB) & 1, wc, kSitePFull))) break;
+      tc_fence_after();
+      const uint32_t stb = tmem + C::TM_ST + (st % C::SB) * C::BMQ;
+#pragma unroll
+      for (int kb = 0; kb < C::BMQ / 16; ++kb)
+        umma_ts_elect(false, tmem + C::TM_DV, stb + half_packed_col<C::BMQ>(kb),
+                      sdesc_sw128(dobuf(st) + hbox * C::BMQ * 128 + kb * 16 * 128, C::BMQ * 128, 1024),
+                      ID_G, (st > 0 || kb > 0) ? 1u : 0u);
+      // dK += dS^T Q[:, part]   (A = dS^T bf16 in TMEM over the dP^T columns)
+      if (!(ok = mbar_wait_warp(bar(C::B_DS + st % C::DB), (st / C::DB) & 1, wc, kSiteDsFull))) break;
+      tc_fence_after();
+      const uint32_t dpb = tmem + C::TM_DPT + (st % C::DB) * C::BMQ;
+#pragma unroll
+      for (int kb = 0; kb < C::BMQ / 16; ++kb)
+        umma_ts_elect(false, tmem + C::TM_DK, dpb + half_packed_col<C::BMQ>(kb),
+                      sdesc_sw128(qbuf(st) + hbox * C::BMQ * 128 + kb * 16 * 128, C::BMQ * 128, 1024),
+                      ID_G, (st > 0 || kb > 0) ? 1u : 0u);
+      tc_commit_elect(bar(C::B_EMPTY + st % C::STAGES));
+      // the next tile's remaining products go after this tile's readers
+      if (nx < nsteps) {
+        if (!EARLY_S && !(ok = issue_st(nx))) break;
+        if (!EARLY_DP) issue_dpt(nx);
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t ID_T = idesc_bf16(128, C::BMQ, false);    // S^T, dP^T: 128 x BMQ
-      constexpr uint32_t ID_G = idesc_bf16(128, C::DH, true);      // dV, dK: 128 x DH, B MN-major
-      bool ok = mbar_wait(bar(C::B_KV), 0, wc, kSiteKFull);
-      for (int st = 0; st < nsteps && ok; ++st) {
-        const int s = st % C::STAGES;
-        if (!(ok = mbar_wait(bar(C::B_FULL + s), (st / C::STAGES) & 1, wc, kSiteQFull))) break;
-        tc_fence_after();
-        const uint32_t qb = sbase + C::SMEM_Q + s * C::QT_BYTES;
-        const uint32_t dob = sbase + C::SMEM_DO + s * C::QT_BYTES;
-#pragma unroll
-        for (int kb = 0; kb < C::D / 16; ++kb) {
-          const int box = kb / 4, off = (kb % 4) * 32;
-          umma_ss<false>(tmem + C::TM_ST,
-                         sdesc_sw128(sbase + C::SMEM_K + box * C::BN * 128 + off, 16, 1024),
-                         sdesc_sw128(qb + box * C::BMQ * 128 + off, 16, 1024), ID_T, kb > 0);
-        }
-#pragma unroll
-        for (int kb = 0; kb < C::D / 16; ++kb) {
-          const int box = kb / 4, off = (kb % 4) * 32;
-          umma_ss<false>(tmem + C::TM_DPT,
-                         sdesc_sw128(sbase + C::SMEM_V + box * C::BN * 128 + off, 16, 1024),
-                         sdesc_sw128(dob + box * C::BMQ * 128 + off, 16, 1024), ID_T, kb > 0);
-        }
-        tc_commit(bar(C::B_SDP));
-        // dV += P^T dO[:, half]   (A = P^T bf16 in TMEM over the S^T columns)
-        if (!(ok = mbar_wait(bar(C::B_P), st & 1, wc, kSitePFull))) break;
-        tc_fence_after();
-        const int hbox = split * (C::DH / 64);
-#pragma unroll
-        for (int kb = 0; kb < C::BMQ / 16; ++kb)
-          umma_ts<false>(tmem + C::TM_DV, tmem + C::TM_ST + kb * 8,
-                         sdesc_sw128(dob + hbox * C::BMQ * 128 + kb * 16 * 128, C::BMQ * 128, 1024),
-                         ID_G, (st > 0 || kb > 0) ? 1u : 0u);
-        // dK += dS^T Q[:, half]   (A = dS^T bf16 in TMEM over the dP^T columns)
-        if (!(ok = mbar_wait(bar(C::B_DS), st & 1, wc, kSiteDsFull))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kb = 0; kb < C::BMQ / 16; ++kb)
-          umma_ts<false>(tmem + C::TM_DK, tmem + C::TM_DPT + kb * 8,
-                         sdesc_sw128(qb + hbox * C::BMQ * 128 + kb * 16 * 128, C::BMQ * 128, 1024),
-                         ID_G, (st > 0 || kb > 0) ? 1u : 0u);
-        tc_commit(bar(C::B_EMPTY + s));
-      }
-      tc_commit(bar(C::B_ACC));
-      tc_commit(bar(C::B_DRAIN));
-      if (!mbar_wait_drain(bar(C::B_DRAIN), 0, wc.timeout_ns))
-        atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
-    }
+    tc_commit_elect(bar(C::B_ACC));
+    tc_commit_elect(bar(C::B_DRAIN));
+    if (!mbar_wait_drain(bar(C::B_DRAIN), 0, wc.timeout_ns) && lane == 0)
+      atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
   } else {
-    // ---------------- compute warps: thread owns key row `row`
-    const int quad = warp & 3;
+    // ---------------- compute warps: thread owns key row `row`, query columns of `half`
+    const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
     const int kv = kt * C::BN + row;
     const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const float LOG2E = 1.4426950408889634f;
     const float sl2 = p.scale * LOG2E;
     bool ok = true;
     for (int st = 0; st < nsteps && ok; ++st) {
       const int s = st % C::STAGES;
       const int qi = i0 + st;
+      const int c_first = qi * C::BMQ + half * C::CH;      // first query of this half
       if (!(ok = mbar_wait(bar(C::B_FULL + s), (st / C::STAGES) & 1, wc, kSiteQFull))) break;
-      if (!(ok = mbar_wait(bar(C::B_SDP), st & 1, wc, kSiteSFull))) break;
+      if (!(ok = mbar_wait(bar(C::B_SFULL + st % C::SB), (st / C::SB) & 1, wc, kSiteSFull))) break;
       tc_fence_after();
-      const float* ls = lse_s + s * C::BMQ;
-      const float* ds_ = dd_s + s * C::BMQ;
-      // P^T row: p_c = 2^(s_c*sl2 - lse_c*log2e), zero where the query may not see this key
-      float pr[C::BMQ];
+      const float* ls = lse_s + s * C::BMQ + half * C::CH;
+      const float* ds_ = dd_s + s * C::BMQ + half * C::CH;
+      const uint32_t stc = lb + C::TM_ST + (st % C::SB) * C::BMQ + half * C::CH;
+      // P^T row segment, zero where the query may not see this key
+      float pr[C::CH];
+      {
+        uint32_t r[C::CH];
+        if constexpr (C::CH == 64) {
+          tmem_ld64(stc, r);
+          tmem_ld_wait64(r);
+        } else {
+          tmem_ld32(stc, r);
+          tmem_ld_wait(r);
+        }
+        exp2_row<C::CH, C::EMU>(r, sl2, ls, pr);
+      }
+      const bool full_vis = (kv < p.N) && (c_first + C::CH <= p.N) &&
+                            (!p.causal || kt * C::BN + C::BN - 1 <= c_first);
+      if (!__all_sync(0xffffffffu, full_vis)) {
 #pragma unroll
-      for (int c0 = 0; c0 < C::BMQ; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(lb + C::TM_ST + c0, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int q = qi * C::BMQ + c0 + i;
-          const bool vis = (q < p.N) && (kv < p.N) && (!p.causal || kv <= q);
-          pr[c0 + i] = vis ? ex2(fmaf(__uint_as_float(r[i]), sl2, -ls[c0 + i] * LOG2E)) : 0.f;
+        for (int i = 0; i < C::CH; ++i) {
+          const int q = c_first + i;
+          if (!((q < p.N) && (kv < p.N) && (!p.causal || kv <= q))) pr[i] = 0.f;
         }
       }
+      {
+        uint32_t w[C::CH / 2];
 #pragma unroll
-      for (int c0 = 0; c0 < C::BMQ; c0 += 64) {
-        uint32_t r[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = pack_bf16x2(pr[c0 + 2 * i], pr[c0 + 2 * i + 1]);
-        tmem_st32(lb + C::TM_ST + c0 / 2, r);
+        for (int i = 0; i < C::CH / 2; ++i) w[i] = pack_bf16x2(pr[2 * i], pr[2 * i + 1]);
+        if constexpr (C::CH == 64)
+          tmem_st32(stc, w);
+        else
+          tmem_st16(stc, w);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive_warp(bar(C::B_P));
-      // dS^T row = P^T * (dP^T - D_q), written as bf16 over the consumed dP^T columns
-#pragma unroll
-      for (int c0 = 0; c0 < C::BMQ; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(lb + C::TM_DPT + c0, r);
-        tmem_ld_wait(r);
-        uint32_t w16[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = pr[c0 + 2 * i] * (__uint_as_float(r[2 * i]) - ds_[c0 + 2 * i]);
-          const float b = pr[c0 + 2 * i + 1] * (__uint_as_float(r[2 * i + 1]) - ds_[c0 + 2 * i + 1]);
-          w16[i] = pack_bf16x2(a, b);
+      mbar_arrive_warp(bar(C::B_P + st % C::SB));
+      // dS^T row segment = P^T (dP^T - D_q), bf16 over this half's dP^T columns
+      if (!(ok = mbar_wait(bar(C::B_DPFULL + st % C::DB), (st / C::DB) & 1, wc, kSiteSFull))) break;
+      tc_fence_after();
+      const uint32_t dpc = lb + C::TM_DPT + (st % C::DB) * C::BMQ + half * C::CH;
+      {
+        uint32_t r[C::CH];
+        if constexpr (C::CH == 64) {
+          tmem_ld64(dpc, r);
+          tmem_ld_wait64(r);
+        } else {
+          tmem_ld32(dpc, r);
+          tmem_ld_wait(r);
         }
-        tmem_st16(lb + C::TM_DPT + c0 / 2, w16);
+        uint32_t w[C::CH / 2];
+#pragma unroll
+        for (int i = 0; i < C::CH / 2; ++i) {
+          float a, b;
+          f2_unpack(f2_mul(f2_pack(pr[2 * i], pr[2 * i + 1]),
+                           f2_add(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                                  f2_pack(-ds_[2 * i], -ds_[2 * i + 1]))),
+                    a, b);
+          w[i] = pack_bf16x2(a, b);
+        }
+        if constexpr (C::CH == 64)
+          tmem_st32(dpc, w);
+        else
+          tmem_st16(dpc, w);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive_warp(bar(C::B_DS));
+      mbar_arrive_warp(bar(C::B_DS + st % C::DB));
     }
-    // epilogue: dV and scale*dK -> bf16 global
+    // epilogue: dV and scale*dK -> bf16 global, this half's DH/2 columns of the row
     if (ok && mbar_wait(bar(C::B_ACC), 0, wc, kSiteDqDone)) {
       tc_fence_after();
       const bool row_ok = kv < p.N;
-      const size_t base = (static_cast<size_t>(bh) * p.N + kv) * C::D + split * C::DH;
+      const size_t base =
+          (static_cast<size_t>(bh) * p.N + kv) * C::D + split * C::DH + half * (C::DH / 2);
       __nv_bfloat16* dvp = reinterpret_cast<__nv_bfloat16*>(p.dv) + base;
       __nv_bfloat16* dkp = reinterpret_cast<__nv_bfloat16*>(p.dk) + base;
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
-        const uint32_t col0 = which == 0 ? C::TM_DV : C::TM_DK;
+        const uint32_t col0 = (which == 0 ? C::TM_DV : C::TM_DK) + half * (C::DH / 2);
         const float mul = which == 0 ? 1.f : p.scale;
         __nv_bfloat16* dst = which == 0 ? dvp : dkp;
 #pragma unroll 1
-        for (int c = 0; c < C::DH; c += 32) {
+        for (int c = 0; c < C::DH / 2; c += 32) {
           uint32_t r[32];
           tmem_ld32(lb + col0 + c, r);
           tmem_ld_wait(r);
@@ -344,19 +460,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
   }
 }
 
 // --------------------------------------------------------------------------- 3. dQ
-template <int D_, int BN_, int STAGES_>
+// One CTA per (head, 128-row query tile).  Q and dO stay in shared memory, dQ
+// accumulates in tensor memory, and the key tiles stream through a ring.  Per key
+// tile j (BN keys): S = Q K_j^T and dP = dO V_j^T on the tensor core; the compute
+// warps form P from the saved logsumexp and dS = P (dP - D) (bf16 over the dP
+// columns); then dQ += dS K_j.  S has SB buffers and dP DB buffers so tile j+1's
+// products overlap the elementwise work on tile j; eight compute warps split the key
+// columns in halves as in the dK/dV pass.
+template <int D_, int BN_, int STAGES_, int SB_, int DB_, int EMU_ = 1>
 struct DqCfg {
   static constexpr int D = D_;
   static constexpr int BN = BN_;        // streamed key rows
   static constexpr int BM = 128;        // query rows of the CTA = TMEM lanes
   static constexpr int STAGES = STAGES_;
+  static constexpr int SB = SB_, DB = DB_;
+  static constexpr int EMU = EMU_;
+  static constexpr int CH = BN / 2;     // key columns per compute warp
   static constexpr int ROW_BYTES = D * 2;
   static constexpr int NBOX = ROW_BYTES / 128;
   static constexpr int QT_BYTES = BM * ROW_BYTES;
@@ -366,15 +492,22 @@ struct DqCfg {
   static constexpr int SMEM_K = 2 * QT_BYTES;
   static constexpr int SMEM_V = SMEM_K + STAGES * KT_BYTES;
   static constexpr int SMEM_BAR = SMEM_V + STAGES * KT_BYTES;
-  static constexpr int B_QDO = 0, B_SDP = 1, B_DS = 2, B_ACC = 3, B_DRAIN = 4, B_FULL = 5,
-                       B_EMPTY = 5 + STAGES, NBARS = 5 + 2 * STAGES;
+  static constexpr int B_QDO = 0, B_ACC = 1, B_DRAIN = 2,
+                       B_SFULL = 3, B_DPFULL = 3 + SB, B_DS = 3 + SB + DB,
+                       B_FULL = 3 + SB + 2 * DB, B_EMPTY = B_FULL + STAGES,
+                       NBARS = B_EMPTY + STAGES;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
-  static constexpr int TM_S = 0, TM_DP = BN, TM_DQ = 2 * BN;
+  static constexpr int TM_S = 0;                 // + b * BN
+  static constexpr int TM_DP = SB * BN;          // + b * BN
+  static constexpr int TM_DQ = (SB + DB) * BN;
   static constexpr int TM_COLS = 512;
-  static constexpr int THREADS = 192;
-  static_assert(2 * BN + D <= TM_COLS, "tensor memory budget");
+  static constexpr int THREADS = 320;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+  static_assert((SB + DB) * BN + D <= TM_COLS, "tensor memory budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+  static_assert(BN % 64 == 0 && CH % 32 == 0, "box and TMEM chunk sizes");
+  static_assert(SB >= 1 && SB <= 2 && DB >= 1 && DB <= 2, "one or two buffers");
 };
 
 template <class C>
@@ -398,11 +531,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int nsteps = p.causal ? min(p.n_kt, ((qt + 1) * C::BM - 1) / C::BN + 1) : p.n_kt;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NBARS; ++i) mbar_init(bar(i), i == C::B_DS ? 4u : 1u);   // 4 warps
+    for (int i = 0; i < C::NBARS; ++i)
+      mbar_init(bar(i), (i >= C::B_DS && i < C::B_DS + C::DB) ? 8u : 1u);   // 8 compute warps
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(tmem_slot), C::TM_COLS);
     tmem_relinquish();
   }
@@ -412,19 +546,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == 0) {
-    if (lane == 0) {
-      bool ok = true;
+  if (warp == C::PRODUCER_WARP) {
+    bool ok = true;
+    if (elect_one()) {
       mbar_arrive_expect_tx(bar(C::B_QDO), 2 * C::QT_BYTES);
       for (int c = 0; c < C::NBOX; ++c) {
         tma_load_3d(sbase + C::SMEM_Q + c * C::BM * 128, &tq, bar(C::B_QDO), c * 64, qt * C::BM, bh);
         tma_load_3d(sbase + C::SMEM_DO + c * C::BM * 128, &tdo, bar(C::B_QDO), c * 64, qt * C::BM, bh);
       }
-      for (int j = 0; j < nsteps && ok; ++j) {
-        const int s = j % C::STAGES;
-        if (j >= C::STAGES &&
-            !(ok = mbar_wait(bar(C::B_EMPTY + s), ((j / C::STAGES) - 1) & 1, wc, kSiteKVEmpty)))
-          break;
+    }
+    __syncwarp();
+    for (int j = 0; j < nsteps && ok; ++j) {
+      const int s = j % C::STAGES;
+      if (j >= C::STAGES &&
+          !(ok = mbar_wait_warp(bar(C::B_EMPTY + s), ((j / C::STAGES) - 1) & 1, wc, kSiteKVEmpty)))
+        break;
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar(C::B_FULL + s), 2 * C::KT_BYTES);
         for (int c = 0; c < C::NBOX; ++c) {
           tma_load_3d(sbase + C::SMEM_K + s * C::KT_BYTES + c * C::BN * 128, &tk, bar(C::B_FULL + s),
@@ -433,56 +570,84 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       c * 64, j * C::BN, bh);
         }
       }
-      if (ok) {
-        for (int j = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); ok && j < nsteps; ++j)
-          ok = mbar_wait(bar(C::B_EMPTY + j % C::STAGES), (j / C::STAGES) & 1, wc, kSiteKVEmpty);
-      } else {
-        mbar_wait_drain(bar(C::B_QDO), 0, 100000000ull);
-        for (int j = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); j < nsteps; ++j)
-          mbar_wait_drain(bar(C::B_FULL + j % C::STAGES), (j / C::STAGES) & 1, 100000000ull);
+      __syncwarp();
+    }
+    if (ok) {
+      for (int j = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); ok && j < nsteps; ++j)
+        ok = mbar_wait_warp(bar(C::B_EMPTY + j % C::STAGES), (j / C::STAGES) & 1, wc, kSiteKVEmpty);
+    } else {
+      mbar_wait_drain(bar(C::B_QDO), 0, 100000000ull);
+      for (int j = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); j < nsteps; ++j)
+        mbar_wait_drain(bar(C::B_FULL + j % C::STAGES), (j / C::STAGES) & 1, 100000000ull);
+    }
+  } else if (warp == C::MMA_WARP) {
+    constexpr uint32_t ID_S = idesc_bf16(128, C::BN, false);
+    constexpr uint32_t ID_Q = idesc_bf16(128, C::D, true);
+    auto kbuf = [&](int j) { return sbase + C::SMEM_K + (j % C::STAGES) * C::KT_BYTES; };
+    auto vbuf = [&](int j) { return sbase + C::SMEM_V + (j % C::STAGES) * C::KT_BYTES; };
+    auto issue_s = [&](int j) -> bool {
+      if (!mbar_wait_warp(bar(C::B_FULL + j % C::STAGES), (j / C::STAGES) & 1, wc, kSiteKFull))
+        return false;
+      tc_fence_after();
+#pragma unroll
+      for (int kb = 0; kb < C::D / 16; ++kb) {
+        const int box = kb / 4, off = (kb % 4) * 32;
+        umma_ss_elect(false, tmem + C::TM_S + (j % C::SB) * C::BN,
+                      sdesc_sw128(sbase + C::SMEM_Q + box * C::BM * 128 + off, 16, 1024),
+                      sdesc_sw128(kbuf(j) + box * C::BN * 128 + off, 16, 1024), ID_S, kb > 0);
+      }
+      tc_commit_elect(bar(C::B_SFULL + j % C::SB));
+      return true;
+    };
+    auto issue_dp = [&](int j) {
+#pragma unroll
+      for (int kb = 0; kb < C::D / 16; ++kb) {
+        const int box = kb / 4, off = (kb % 4) * 32;
+        umma_ss_elect(false, tmem + C::TM_DP + (j % C::DB) * C::BN,
+                      sdesc_sw128(sbase + C::SMEM_DO + box * C::BM * 128 + off, 16, 1024),
+                      sdesc_sw128(vbuf(j) + box * C::BN * 128 + off, 16, 1024), ID_S, kb > 0);
+      }
+      tc_commit_elect(bar(C::B_DPFULL + j % C::DB));
+    };
+    // S(j+1) may run ahead of dQ(j): its buffer's last reader, the compute warps'
+    // load of S(j+1-SB), happened before they released dS(j+1-SB).  dP(j+1) has to
+    // follow dQ(j) unless it has a second buffer.
+    constexpr bool EARLY_S = C::SB == 2 && C::STAGES >= 2;
+    constexpr bool EARLY_DP = EARLY_S && C::DB == 2;
+    bool ok = mbar_wait_warp(bar(C::B_QDO), 0, wc, kSiteQFull);
+    if (ok && nsteps > 0) {
+      ok = issue_s(0);
+      if (ok) issue_dp(0);
+    }
+    for (int j = 0; j < nsteps && ok; ++j) {
+      const int nx = j + 1;
+      if (EARLY_S && nx < nsteps) {
+        // S(nx) overwrites the buffer S(nx - 2) was loaded from: that load preceded
+        // dS(nx - 2), which this warp waited for one iteration ago
+        if (!(ok = issue_s(nx))) break;
+        if (EARLY_DP) issue_dp(nx);
+      }
+      if (!(ok = mbar_wait_warp(bar(C::B_DS + j % C::DB), (j / C::DB) & 1, wc, kSiteDsFull))) break;
+      tc_fence_after();
+      // dQ += dS K_j: A = dS (query rows x key cols) bf16 in TMEM, B = K_j MN-major
+      const uint32_t dpb = tmem + C::TM_DP + (j % C::DB) * C::BN;
+#pragma unroll
+      for (int kb = 0; kb < C::BN / 16; ++kb)
+        umma_ts_elect(false, tmem + C::TM_DQ, dpb + half_packed_col<C::BN>(kb),
+                      sdesc_sw128(kbuf(j) + kb * 16 * 128, C::BN * 128, 1024), ID_Q,
+                      (j > 0 || kb > 0) ? 1u : 0u);
+      tc_commit_elect(bar(C::B_EMPTY + j % C::STAGES));
+      if (nx < nsteps) {
+        if (!EARLY_S && !(ok = issue_s(nx))) break;
+        if (!EARLY_DP) issue_dp(nx);
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t ID_S = idesc_bf16(128, C::BN, false);
-      constexpr uint32_t ID_Q = idesc_bf16(128, C::D, true);
-      bool ok = mbar_wait(bar(C::B_QDO), 0, wc, kSiteQFull);
-      for (int j = 0; j < nsteps && ok; ++j) {
-        const int s = j % C::STAGES;
-        if (!(ok = mbar_wait(bar(C::B_FULL + s), (j / C::STAGES) & 1, wc, kSiteKFull))) break;
-        tc_fence_after();
-        const uint32_t kb_ = sbase + C::SMEM_K + s * C::KT_BYTES;
-        const uint32_t vb_ = sbase + C::SMEM_V + s * C::KT_BYTES;
-#pragma unroll
-        for (int kb = 0; kb < C::D / 16; ++kb) {
-          const int box = kb / 4, off = (kb % 4) * 32;
-          umma_ss<false>(tmem + C::TM_S, sdesc_sw128(sbase + C::SMEM_Q + box * C::BM * 128 + off, 16, 1024),
-                         sdesc_sw128(kb_ + box * C::BN * 128 + off, 16, 1024), ID_S, kb > 0);
-        }
-#pragma unroll
-        for (int kb = 0; kb < C::D / 16; ++kb) {
-          const int box = kb / 4, off = (kb % 4) * 32;
-          umma_ss<false>(tmem + C::TM_DP, sdesc_sw128(sbase + C::SMEM_DO + box * C::BM * 128 + off, 16, 1024),
-                         sdesc_sw128(vb_ + box * C::BN * 128 + off, 16, 1024), ID_S, kb > 0);
-        }
-        tc_commit(bar(C::B_SDP));
-        if (!(ok = mbar_wait(bar(C::B_DS), j & 1, wc, kSiteDsFull))) break;
-        tc_fence_after();
-        // dQ += dS K_j: A = dS (query rows x key cols) bf16 in TMEM, B = K_j MN-major
-#pragma unroll
-        for (int kb = 0; kb < C::BN / 16; ++kb)
-          umma_ts<false>(tmem + C::TM_DQ, tmem + C::TM_DP + kb * 8,
-                         sdesc_sw128(kb_ + kb * 16 * 128, C::BN * 128, 1024), ID_Q,
-                         (j > 0 || kb > 0) ? 1u : 0u);
-        tc_commit(bar(C::B_EMPTY + s));
-      }
-      tc_commit(bar(C::B_ACC));
-      tc_commit(bar(C::B_DRAIN));
-      if (!mbar_wait_drain(bar(C::B_DRAIN), 0, wc.timeout_ns))
-        atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
-    }
+    tc_commit_elect(bar(C::B_ACC));
+    tc_commit_elect(bar(C::B_DRAIN));
+    if (!mbar_wait_drain(bar(C::B_DRAIN), 0, wc.timeout_ns) && lane == 0)
+      atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
   } else {
-    const int quad = warp & 3;
+    const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
     const int q = qt * C::BM + row;
     const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
@@ -493,44 +658,70 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const float dq_i = row_ok ? p.drow[static_cast<size_t>(bh) * p.N + q] : 0.f;
     bool ok = true;
     for (int j = 0; j < nsteps && ok; ++j) {
-      if (!(ok = mbar_wait(bar(C::B_SDP), j & 1, wc, kSiteSFull))) break;
+      const int k_first = j * C::BN + half * C::CH;          // first key of this half
+      if (!(ok = mbar_wait(bar(C::B_SFULL + j % C::SB), (j / C::SB) & 1, wc, kSiteSFull))) break;
       tc_fence_after();
-      float pr[C::BN];
+      float pr[C::CH];
+      {
+        const uint32_t sc = lb + C::TM_S + (j % C::SB) * C::BN + half * C::CH;
+        uint32_t r[C::CH];
+        if constexpr (C::CH == 64) {
+          tmem_ld64(sc, r);
+          tmem_ld_wait64(r);
+        } else {
+          tmem_ld32(sc, r);
+          tmem_ld_wait(r);
+        }
+        exp2_row<C::CH, C::EMU>(r, sl2, lse2, pr);
+      }
+      const bool full_vis = row_ok && (k_first + C::CH <= p.N) &&
+                            (!p.causal || k_first + C::CH - 1 <= qt * C::BM);
+      if (!__all_sync(0xffffffffu, full_vis)) {
 #pragma unroll
-      for (int c0 = 0; c0 < C::BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(lb + C::TM_S + c0, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int kv = j * C::BN + c0 + i;
-          const bool vis = row_ok && (kv < p.N) && (!p.causal || kv <= q);
-          pr[c0 + i] = vis ? ex2(fmaf(__uint_as_float(r[i]), sl2, -lse2)) : 0.f;
+        for (int i = 0; i < C::CH; ++i) {
+          const int kv = k_first + i;
+          if (!(row_ok && (kv < p.N) && (!p.causal || kv <= q))) pr[i] = 0.f;
         }
       }
+      if (!(ok = mbar_wait(bar(C::B_DPFULL + j % C::DB), (j / C::DB) & 1, wc, kSiteSFull))) break;
+      tc_fence_after();
+      {
+        const uint32_t dc = lb + C::TM_DP + (j % C::DB) * C::BN + half * C::CH;
+        uint32_t r[C::CH];
+        if constexpr (C::CH == 64) {
+          tmem_ld64(dc, r);
+          tmem_ld_wait64(r);
+        } else {
+          tmem_ld32(dc, r);
+          tmem_ld_wait(r);
+        }
+        const uint64_t nd2 = f2_pack(-dq_i, -dq_i);
+        uint32_t w[C::CH / 2];
 #pragma unroll
-      for (int c0 = 0; c0 < C::BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(lb + C::TM_DP + c0, r);
-        tmem_ld_wait(r);
-        uint32_t w16[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w16[i] = pack_bf16x2(pr[c0 + 2 * i] * (__uint_as_float(r[2 * i]) - dq_i),
-                               pr[c0 + 2 * i + 1] * (__uint_as_float(r[2 * i + 1]) - dq_i));
-        tmem_st16(lb + C::TM_DP + c0 / 2, w16);
+        for (int i = 0; i < C::CH / 2; ++i) {
+          float a, b;
+          f2_unpack(f2_mul(f2_pack(pr[2 * i], pr[2 * i + 1]),
+                           f2_add(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), nd2)),
+                    a, b);
+          w[i] = pack_bf16x2(a, b);
+        }
+        if constexpr (C::CH == 64)
+          tmem_st32(dc, w);
+        else
+          tmem_st16(dc, w);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive_warp(bar(C::B_DS));
+      mbar_arrive_warp(bar(C::B_DS + j % C::DB));
     }
     if (ok && mbar_wait(bar(C::B_ACC), 0, wc, kSiteDqDone)) {
       tc_fence_after();
-      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(bh) * p.N + q) * C::D;
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.dq) +
+                           (static_cast<size_t>(bh) * p.N + q) * C::D + half * (C::D / 2);
 #pragma unroll 1
-      for (int c = 0; c < C::D; c += 32) {
+      for (int c = 0; c < C::D / 2; c += 32) {
         uint32_t r[32];
-        tmem_ld32(lb + C::TM_DQ + c, r);
+        tmem_ld32(lb + C::TM_DQ + half * (C::D / 2) + c, r);
         tmem_ld_wait(r);
         uint32_t pk[16];
 #pragma unroll
@@ -547,7 +738,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
   }

@@ -279,36 +279,8 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint3
     atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
 }
 
-// ---------------------------------------------------------------- software exp2
-// 2^x for a pair of fp32 values on the FMA/ALU pipes instead of the special-function
-// unit (the issoh.co.jp page, section FA4のB200で1613TFLOPs…, on why Blackwell needs
-// part of the exponentials in software).  Cody-Waite reduction x = n + f with
-// n = rint(x) (added to 1.5*2^23 so n lands in the low mantissa bits) and
-// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial with minimax relative error 7.5e-5
-// (coefficients from csrc/fit_exp2_poly.py); 2^n by adding n << 23 to the
-// exponent field.  x is clamped at -126 (the result there, about 1.2e-38, stands in
-// for anything smaller), so the exponent field never underflows; valid for x <= 127.
-// Only used on tiles with no masked scores, so a masked -inf never reaches it.
-__device__ __forceinline__ uint64_t ex2_poly_pair(uint64_t x2) {
-  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f,
-                  kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
-  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-  float xa, xb;
-  f2_unpack(x2, xa, xb);
-  const uint64_t x = f2_pack(fmaxf(xa, -126.f), fmaxf(xb, -126.f));
-  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
-  const uint64_t nf = f2_add(t, f2_pack(-kRound, -kRound));
-  const uint64_t f = f2_fma(nf, f2_pack(-1.f, -1.f), x);
-  uint64_t p = f2_fma(f2_pack(kC3, kC3), f, f2_pack(kC2, kC2));
-  p = f2_fma(p, f, f2_pack(kC1, kC1));
-  p = f2_fma(p, f, f2_pack(kC0, kC0));
-  float pa, pb, ta, tb;
-  f2_unpack(p, pa, pb);
-  f2_unpack(t, ta, tb);
-  const uint32_t ra = __float_as_uint(pa) + (__float_as_uint(ta) << 23);
-  const uint32_t rb = __float_as_uint(pb) + (__float_as_uint(tb) << 23);
-  return f2_pack(__uint_as_float(ra), __uint_as_float(rb));
-}
+// ---------------------------------------------------------------- exp2 variants
+// ex2_poly_pair (software 2^x on the FMA pipe) lives in sm100_ptx.cuh.
 
 // 2^x for a pair of fp32 values on the special-function unit in half precision:
 // one ex2.approx.f16x2 for both.  The argument is rounded to f16 (relative 2^-11,
