@@ -323,12 +323,18 @@ using FwdD128 = FwdPick<FA_FWD_D128_KIND, 128, false>;
 using FwdF8D128 = FwdPick<FA_FWD_F8_KIND, 128, true>;
 using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_EMU>;
 
-using DkdvD64 = DkdvCfg<64, 64, 128, 3, 2, 1>;
-using DkdvD128 = DkdvCfg<128, 128, 64, 3, 2, 2>;
-using DkdvD256 = DkdvCfg<256, 128, 64, 1, 2, 2>;
-using DqD64 = DqCfg<64, 128, 3, 2, 1>;
-using DqD128 = DqCfg<128, 128, 2, 2, 1>;
-using DqD256 = DqCfg<256, 64, 1, 2, 2>;
+#ifndef FA_BWD_EMU
+#define FA_BWD_EMU 1
+#endif
+#ifndef FA_BWD_D64_STAGES
+#define FA_BWD_D64_STAGES 3
+#endif
+using DkdvD64 = DkdvCfg<64, 64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU>;
+using DkdvD128 = DkdvCfg<128, 128, 64, 3, 3, 2, 2, FA_BWD_EMU>;
+using DkdvD256 = DkdvCfg<256, 128, 64, 2, 1, 2, 2, FA_BWD_EMU>;
+using DqD64 = DqCfg<64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU>;
+using DqD128 = DqCfg<128, 128, 2, 2, 2, 1, FA_BWD_EMU>;
+using DqD256 = DqCfg<256, 64, 2, 1, 2, 2, FA_BWD_EMU>;
 
 template <class CK, class CQ>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,

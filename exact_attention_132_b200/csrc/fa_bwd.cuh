@@ -85,18 +85,21 @@ __global__ void __launch_bounds__(256) fa_bwd_rowdot(const __nv_bfloat16* __rest
 //   dS^T = P^T (dP^T - D_i)                             (compute warps, bf16 over dP^T)
 //   dK += dS^T Q_i                                      (tensor core, A = dS^T from TMEM)
 // S^T and dP^T have SB / DB buffers, so the products of tile i+1 run on the tensor
-// core while the compute warps work on tile i.  Eight compute warps: two per TMEM lane
+// core while the compute warps work on tile i.  Q_i (with lse_i) and dO_i (with D_i)
+// stream through rings of their own, QST and OST deep: dO_i is free once dV has read
+// it, Q_i only after dK, so at d = 256, where shared memory holds three query-tile
+// slots, Q gets two and dO one.  Eight compute warps: two per TMEM lane
 // quadrant, each owning half of the BMQ query columns (P needs no row reduction, so
 // the halves never talk to each other).  Each half writes its bf16 P^T / dS^T into
 // the first half of its own column range.
-template <int D_, int DH_, int BMQ_, int STAGES_, int SB_, int DB_, int EMU_ = 1>
+template <int D_, int DH_, int BMQ_, int QST_, int OST_, int SB_, int DB_, int EMU_ = 1>
 struct DkdvCfg {
   static constexpr int D = D_;          // head dim (contraction of S^T and dP^T)
   static constexpr int DH = DH_;        // columns of dK/dV this CTA produces
   static constexpr int NSPLIT = D / DH;
   static constexpr int BMQ = BMQ_;      // query rows per streamed tile
   static constexpr int BN = 128;        // key rows of the CTA = TMEM lanes
-  static constexpr int STAGES = STAGES_;
+  static constexpr int QST = QST_, OST = OST_;
   static constexpr int SB = SB_, DB = DB_;
   static constexpr int EMU = EMU_;      // software exp2 share, in quarters
   static constexpr int CH = BMQ / 2;    // query columns per compute warp
@@ -107,15 +110,20 @@ struct DkdvCfg {
   static constexpr int SMEM_K = 0;
   static constexpr int SMEM_V = KT_BYTES;
   static constexpr int SMEM_Q = 2 * KT_BYTES;
-  static constexpr int SMEM_DO = SMEM_Q + STAGES * QT_BYTES;
-  static constexpr int SMEM_LSE = SMEM_DO + STAGES * QT_BYTES;    // [STAGES][BMQ] fp32
-  static constexpr int SMEM_DD = SMEM_LSE + STAGES * BMQ * 4;     // [STAGES][BMQ] fp32
-  static constexpr int SMEM_BAR = SMEM_DD + STAGES * BMQ * 4;
+  static constexpr int SMEM_DO = SMEM_Q + QST * QT_BYTES;
+  static constexpr int SMEM_LSE = SMEM_DO + OST * QT_BYTES;       // [QST][BMQ] fp32
+  // D_i has one slot more than dO: the producer refills a slot once dV has read the dO
+  // tile OST steps back, which can precede the compute warps' last use of that step's
+  // D_i by one step
+  static constexpr int DDR = OST + 1;
+  static constexpr int SMEM_DD = SMEM_LSE + QST * BMQ * 4;        // [DDR][BMQ] fp32
+  static constexpr int SMEM_BAR = SMEM_DD + DDR * BMQ * 4;
   static constexpr int B_KV = 0, B_ACC = 1, B_DRAIN = 2,
                        B_SFULL = 3, B_P = 3 + SB,                   // + buffer
                        B_DPFULL = 3 + 2 * SB, B_DS = 3 + 2 * SB + DB,
-                       B_FULL = 3 + 2 * SB + 2 * DB, B_EMPTY = B_FULL + STAGES,
-                       NBARS = B_EMPTY + STAGES;
+                       B_QFULL = 3 + 2 * SB + 2 * DB, B_QEMPTY = B_QFULL + QST,
+                       B_OFULL = B_QEMPTY + QST, B_OEMPTY = B_OFULL + OST,
+                       NBARS = B_OEMPTY + OST;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
   static constexpr int TM_ST = 0;                        // + b * BMQ
@@ -233,48 +241,84 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     }
     __syncwarp();
-    for (int st = 0; st < nsteps && ok; ++st) {
-      const int s = st % C::STAGES;
-      const int qi = i0 + st;
-      if (st >= C::STAGES &&
-          !(ok = mbar_wait_warp(bar(C::B_EMPTY + s), ((st / C::STAGES) - 1) & 1, wc, kSiteKVEmpty)))
-        break;
-      for (int c = lane; c < C::BMQ; c += 32) {
-        const int q = qi * C::BMQ + c;
+    // Q_i (and lse_i) into its ring, then dO_i (and D_i) into its own.  Q_i first: the
+    // MMA warp may ask for Q_i (an early S^T) before it has issued the dV product that
+    // frees the dO slot.  lse and D of the next tile are fetched into registers one
+    // step ahead, so their global-load latency overlaps this step's waits.
+    constexpr int PL = C::BMQ / 32;          // values per lane
+    float lse_n[PL], dd_n[PL];
+    auto fetch = [&](int st) {
+#pragma unroll
+      for (int i = 0; i < PL; ++i) {
+        const int q = (i0 + st) * C::BMQ + lane + 32 * i;
         const bool in = q < p.N;
-        lse_s[s * C::BMQ + c] = in ? p.lse[static_cast<size_t>(bh) * p.N + q] * LOG2E : 0.f;
-        dd_s[s * C::BMQ + c] = in ? p.drow[static_cast<size_t>(bh) * p.N + q] : 0.f;
+        lse_n[i] = in ? p.lse[static_cast<size_t>(bh) * p.N + q] * LOG2E : 0.f;
+        dd_n[i] = in ? p.drow[static_cast<size_t>(bh) * p.N + q] : 0.f;
       }
+    };
+    if (nsteps > 0) fetch(0);
+    int nq = 0, no = 0;                      // tiles issued per ring
+    for (int st = 0; st < nsteps && ok; ++st) {
+      const int qi = i0 + st;
+      const int so = st % C::OST, sq = st % C::QST;
+      float lse_c[PL], dd_c[PL];
+#pragma unroll
+      for (int i = 0; i < PL; ++i) {
+        lse_c[i] = lse_n[i];
+        dd_c[i] = dd_n[i];
+      }
+      if (st + 1 < nsteps) fetch(st + 1);
+      if (st >= C::QST &&
+          !(ok = mbar_wait_warp(bar(C::B_QEMPTY + sq), ((st / C::QST) - 1) & 1, wc, kSiteKVEmpty)))
+        break;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) lse_s[sq * C::BMQ + lane + 32 * i] = lse_c[i];
       __syncwarp();
       if (elect_one()) {
-        mbar_arrive_expect_tx(bar(C::B_FULL + s), 2 * C::QT_BYTES);
-        for (int c = 0; c < C::NBOX; ++c) {
-          tma_load_3d(sbase + C::SMEM_Q + s * C::QT_BYTES + c * C::BMQ * 128, &tq,
-                      bar(C::B_FULL + s), c * 64, qi * C::BMQ, bh);
-          tma_load_3d(sbase + C::SMEM_DO + s * C::QT_BYTES + c * C::BMQ * 128, &tdo,
-                      bar(C::B_FULL + s), c * 64, qi * C::BMQ, bh);
-        }
+        mbar_arrive_expect_tx(bar(C::B_QFULL + sq), C::QT_BYTES);
+        for (int c = 0; c < C::NBOX; ++c)
+          tma_load_3d(sbase + C::SMEM_Q + sq * C::QT_BYTES + c * C::BMQ * 128, &tq,
+                      bar(C::B_QFULL + sq), c * 64, qi * C::BMQ, bh);
       }
       __syncwarp();
+      ++nq;
+      if (st >= C::OST &&
+          !(ok = mbar_wait_warp(bar(C::B_OEMPTY + so), ((st / C::OST) - 1) & 1, wc, kSiteKVEmpty)))
+        break;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) dd_s[(st % C::DDR) * C::BMQ + lane + 32 * i] = dd_c[i];
+      __syncwarp();
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(C::B_OFULL + so), C::QT_BYTES);
+        for (int c = 0; c < C::NBOX; ++c)
+          tma_load_3d(sbase + C::SMEM_DO + so * C::QT_BYTES + c * C::BMQ * 128, &tdo,
+                      bar(C::B_OFULL + so), c * 64, qi * C::BMQ, bh);
+      }
+      __syncwarp();
+      ++no;
     }
     if (ok) {
-      for (int st = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); ok && st < nsteps; ++st)
-        ok = mbar_wait_warp(bar(C::B_EMPTY + st % C::STAGES), (st / C::STAGES) & 1, wc, kSiteKVEmpty);
+      for (int st = (nsteps > C::OST ? nsteps - C::OST : 0); ok && st < nsteps; ++st)
+        ok = mbar_wait_warp(bar(C::B_OEMPTY + st % C::OST), (st / C::OST) & 1, wc, kSiteKVEmpty);
+      for (int st = (nsteps > C::QST ? nsteps - C::QST : 0); ok && st < nsteps; ++st)
+        ok = mbar_wait_warp(bar(C::B_QEMPTY + st % C::QST), (st / C::QST) & 1, wc, kSiteKVEmpty);
     } else {
       mbar_wait_drain(bar(C::B_KV), 0, 100000000ull);
-      for (int st = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); st < nsteps; ++st)
-        mbar_wait_drain(bar(C::B_FULL + st % C::STAGES), (st / C::STAGES) & 1, 100000000ull);
+      for (int st = (no > C::OST ? no - C::OST : 0); st < no; ++st)
+        mbar_wait_drain(bar(C::B_OFULL + st % C::OST), (st / C::OST) & 1, 100000000ull);
+      for (int st = (nq > C::QST ? nq - C::QST : 0); st < nq; ++st)
+        mbar_wait_drain(bar(C::B_QFULL + st % C::QST), (st / C::QST) & 1, 100000000ull);
     }
   } else if (warp == C::MMA_WARP) {
     // ---------------- MMA issuer (whole warp, one elected lane issues)
     constexpr uint32_t ID_T = idesc_bf16(128, C::BMQ, false);    // S^T, dP^T: 128 x BMQ
     constexpr uint32_t ID_G = idesc_bf16(128, C::DH, true);      // dV, dK: 128 x DH, B MN-major
     const int hbox = split * (C::DH / 64);
-    auto qbuf = [&](int st) { return sbase + C::SMEM_Q + (st % C::STAGES) * C::QT_BYTES; };
-    auto dobuf = [&](int st) { return sbase + C::SMEM_DO + (st % C::STAGES) * C::QT_BYTES; };
+    auto qbuf = [&](int st) { return sbase + C::SMEM_Q + (st % C::QST) * C::QT_BYTES; };
+    auto dobuf = [&](int st) { return sbase + C::SMEM_DO + (st % C::OST) * C::QT_BYTES; };
     // S^T(st) = K Q^T and, with it or later, dP^T(st) = V dO^T
     auto issue_st = [&](int st) -> bool {
-      if (!mbar_wait_warp(bar(C::B_FULL + st % C::STAGES), (st / C::STAGES) & 1, wc, kSiteQFull))
+      if (!mbar_wait_warp(bar(C::B_QFULL + st % C::QST), (st / C::QST) & 1, wc, kSiteQFull))
         return false;
       tc_fence_after();
 #pragma unroll
@@ -287,7 +331,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_commit_elect(bar(C::B_SFULL + st % C::SB));
       return true;
     };
-    auto issue_dpt = [&](int st) {
+    auto issue_dpt = [&](int st) -> bool {
+      if (!mbar_wait_warp(bar(C::B_OFULL + st % C::OST), (st / C::OST) & 1, wc, kSiteQFull))
+        return false;
+      tc_fence_after();
 #pragma unroll
       for (int kb = 0; kb < C::D / 16; ++kb) {
         const int box = kb / 4, off = (kb % 4) * 32;
@@ -296,23 +343,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       sdesc_sw128(dobuf(st) + box * C::BMQ * 128 + off, 16, 1024), ID_T, kb > 0);
       }
       tc_commit_elect(bar(C::B_DPFULL + st % C::DB));
+      return true;
     };
     bool ok = mbar_wait_warp(bar(C::B_KV), 0, wc, kSiteKFull);
     // prologue: tile 0's products, then tile 1's where the buffers allow
     if (ok && nsteps > 0) {
-      ok = issue_st(0);
-      if (ok) issue_dpt(0);
+      ok = issue_st(0) && issue_dpt(0);
     }
     // Tile st+1's products go ahead of tile st's gradient products when they have a
-    // buffer of their own and their query tile can already be resident (a second ring
-    // stage); otherwise they follow them.
-    constexpr bool EARLY_S = C::SB == 2 && C::STAGES >= 2;
-    constexpr bool EARLY_DP = EARLY_S && C::DB == 2;
+    // buffer of their own and their operand tile can already be resident (a second
+    // ring slot); otherwise they follow them.
+    constexpr bool EARLY_S = C::SB == 2 && C::QST >= 2;
+    constexpr bool EARLY_DP = EARLY_S && C::DB == 2 && C::OST >= 2;
     for (int st = 0; st < nsteps && ok; ++st) {
       const int nx = st + 1;
       // S^T(st+1) into the other buffer (its last reader, dV(st+1-SB), is issued)
       if (EARLY_S && nx < nsteps && !(ok = issue_st(nx))) break;
-      if (EARLY_DP && nx < nsteps) issue_dpt(nx);
+      if (EARLY_DP && nx < nsteps && !(ok = issue_dpt(nx))) break;
       // dV += P^T dO[:, part]   (A = P^T bf16 in TMEM over the S^T columns)
       if (!(ok = mbar_wait_warp(bar(C::B_P + st % C::SB), (st / C::SB) & 1, wc, kSitePFull))) break;
       tc_fence_after();
@@ -322,6 +369,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         umma_ts_elect(false, tmem + C::TM_DV, stb + half_packed_col<C::BMQ>(kb),
                       sdesc_sw128(dobuf(st) + hbox * C::BMQ * 128 + kb * 16 * 128, C::BMQ * 128, 1024),
                       ID_G, (st > 0 || kb > 0) ? 1u : 0u);
+      tc_commit_elect(bar(C::B_OEMPTY + st % C::OST));     // dP^T(st) and dV(st) read dO(st)
       // dK += dS^T Q[:, part]   (A = dS^T bf16 in TMEM over the dP^T columns)
       if (!(ok = mbar_wait_warp(bar(C::B_DS + st % C::DB), (st / C::DB) & 1, wc, kSiteDsFull))) break;
       tc_fence_after();
@@ -331,11 +379,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         umma_ts_elect(false, tmem + C::TM_DK, dpb + half_packed_col<C::BMQ>(kb),
                       sdesc_sw128(qbuf(st) + hbox * C::BMQ * 128 + kb * 16 * 128, C::BMQ * 128, 1024),
                       ID_G, (st > 0 || kb > 0) ? 1u : 0u);
-      tc_commit_elect(bar(C::B_EMPTY + st % C::STAGES));
+      tc_commit_elect(bar(C::B_QEMPTY + st % C::QST));     // S^T(st) and dK(st) read Q(st)
       // the next tile's remaining products go after this tile's readers
       if (nx < nsteps) {
         if (!EARLY_S && !(ok = issue_st(nx))) break;
-        if (!EARLY_DP) issue_dpt(nx);
+        if (!EARLY_DP && !(ok = issue_dpt(nx))) break;
       }
     }
     tc_commit_elect(bar(C::B_ACC));
@@ -351,14 +399,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const float sl2 = p.scale * LOG2E;
     bool ok = true;
     for (int st = 0; st < nsteps && ok; ++st) {
-      const int s = st % C::STAGES;
       const int qi = i0 + st;
       const int c_first = qi * C::BMQ + half * C::CH;      // first query of this half
-      if (!(ok = mbar_wait(bar(C::B_FULL + s), (st / C::STAGES) & 1, wc, kSiteQFull))) break;
+      // lse_i and D_i come with their rings' tiles (and are in place once they are)
+      if (!(ok = mbar_wait(bar(C::B_QFULL + st % C::QST), (st / C::QST) & 1, wc, kSiteQFull))) break;
+      if (!(ok = mbar_wait(bar(C::B_OFULL + st % C::OST), (st / C::OST) & 1, wc, kSiteQFull))) break;
+      const float* dd = dd_s + (st % C::DDR) * C::BMQ + half * C::CH;
       if (!(ok = mbar_wait(bar(C::B_SFULL + st % C::SB), (st / C::SB) & 1, wc, kSiteSFull))) break;
       tc_fence_after();
-      const float* ls = lse_s + s * C::BMQ + half * C::CH;
-      const float* ds_ = dd_s + s * C::BMQ + half * C::CH;
+      const float* ls = lse_s + (st % C::QST) * C::BMQ + half * C::CH;
       const uint32_t stc = lb + C::TM_ST + (st % C::SB) * C::BMQ + half * C::CH;
       // P^T row segment, zero where the query may not see this key
       float pr[C::CH];
@@ -413,7 +462,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           float a, b;
           f2_unpack(f2_mul(f2_pack(pr[2 * i], pr[2 * i + 1]),
                            f2_add(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
-                                  f2_pack(-ds_[2 * i], -ds_[2 * i + 1]))),
+                                  f2_pack(-dd[2 * i], -dd[2 * i + 1]))),
                     a, b);
           w[i] = pack_bf16x2(a, b);
         }
@@ -473,13 +522,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // warps form P from the saved logsumexp and dS = P (dP - D) (bf16 over the dP
 // columns); then dQ += dS K_j.  S has SB buffers and dP DB buffers so tile j+1's
 // products overlap the elementwise work on tile j; eight compute warps split the key
-// columns in halves as in the dK/dV pass.
-template <int D_, int BN_, int STAGES_, int SB_, int DB_, int EMU_ = 1>
+// columns in halves as in the dK/dV pass.  K_j and V_j have rings of their own (KST,
+// VST deep): V_j is free as soon as dP has read it, K_j only after dQ.
+template <int D_, int BN_, int KST_, int VST_, int SB_, int DB_, int EMU_ = 1>
 struct DqCfg {
   static constexpr int D = D_;
   static constexpr int BN = BN_;        // streamed key rows
   static constexpr int BM = 128;        // query rows of the CTA = TMEM lanes
-  static constexpr int STAGES = STAGES_;
+  static constexpr int KST = KST_, VST = VST_;
   static constexpr int SB = SB_, DB = DB_;
   static constexpr int EMU = EMU_;
   static constexpr int CH = BN / 2;     // key columns per compute warp
@@ -490,12 +540,13 @@ struct DqCfg {
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_DO = QT_BYTES;
   static constexpr int SMEM_K = 2 * QT_BYTES;
-  static constexpr int SMEM_V = SMEM_K + STAGES * KT_BYTES;
-  static constexpr int SMEM_BAR = SMEM_V + STAGES * KT_BYTES;
+  static constexpr int SMEM_V = SMEM_K + KST * KT_BYTES;
+  static constexpr int SMEM_BAR = SMEM_V + VST * KT_BYTES;
   static constexpr int B_QDO = 0, B_ACC = 1, B_DRAIN = 2,
                        B_SFULL = 3, B_DPFULL = 3 + SB, B_DS = 3 + SB + DB,
-                       B_FULL = 3 + SB + 2 * DB, B_EMPTY = B_FULL + STAGES,
-                       NBARS = B_EMPTY + STAGES;
+                       B_KFULL = 3 + SB + 2 * DB, B_KEMPTY = B_KFULL + KST,
+                       B_VFULL = B_KEMPTY + KST, B_VEMPTY = B_VFULL + VST,
+                       NBARS = B_VEMPTY + VST;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
   static constexpr int TM_S = 0;                 // + b * BN
@@ -556,37 +607,53 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     }
     __syncwarp();
+    // K_j then V_j, each into its own ring (an early S(j) needs K_j before the dP
+    // product that frees V's slot is issued)
+    int nk = 0, nv = 0;
     for (int j = 0; j < nsteps && ok; ++j) {
-      const int s = j % C::STAGES;
-      if (j >= C::STAGES &&
-          !(ok = mbar_wait_warp(bar(C::B_EMPTY + s), ((j / C::STAGES) - 1) & 1, wc, kSiteKVEmpty)))
+      const int sk = j % C::KST, sv = j % C::VST;
+      if (j >= C::KST &&
+          !(ok = mbar_wait_warp(bar(C::B_KEMPTY + sk), ((j / C::KST) - 1) & 1, wc, kSiteKVEmpty)))
         break;
       if (elect_one()) {
-        mbar_arrive_expect_tx(bar(C::B_FULL + s), 2 * C::KT_BYTES);
-        for (int c = 0; c < C::NBOX; ++c) {
-          tma_load_3d(sbase + C::SMEM_K + s * C::KT_BYTES + c * C::BN * 128, &tk, bar(C::B_FULL + s),
-                      c * 64, j * C::BN, bh);
-          tma_load_3d(sbase + C::SMEM_V + s * C::KT_BYTES + c * C::BN * 128, &tv, bar(C::B_FULL + s),
-                      c * 64, j * C::BN, bh);
-        }
+        mbar_arrive_expect_tx(bar(C::B_KFULL + sk), C::KT_BYTES);
+        for (int c = 0; c < C::NBOX; ++c)
+          tma_load_3d(sbase + C::SMEM_K + sk * C::KT_BYTES + c * C::BN * 128, &tk,
+                      bar(C::B_KFULL + sk), c * 64, j * C::BN, bh);
       }
       __syncwarp();
+      ++nk;
+      if (j >= C::VST &&
+          !(ok = mbar_wait_warp(bar(C::B_VEMPTY + sv), ((j / C::VST) - 1) & 1, wc, kSiteKVEmpty)))
+        break;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(C::B_VFULL + sv), C::KT_BYTES);
+        for (int c = 0; c < C::NBOX; ++c)
+          tma_load_3d(sbase + C::SMEM_V + sv * C::KT_BYTES + c * C::BN * 128, &tv,
+                      bar(C::B_VFULL + sv), c * 64, j * C::BN, bh);
+      }
+      __syncwarp();
+      ++nv;
     }
     if (ok) {
-      for (int j = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); ok && j < nsteps; ++j)
-        ok = mbar_wait_warp(bar(C::B_EMPTY + j % C::STAGES), (j / C::STAGES) & 1, wc, kSiteKVEmpty);
+      for (int j = (nsteps > C::KST ? nsteps - C::KST : 0); ok && j < nsteps; ++j)
+        ok = mbar_wait_warp(bar(C::B_KEMPTY + j % C::KST), (j / C::KST) & 1, wc, kSiteKVEmpty);
+      for (int j = (nsteps > C::VST ? nsteps - C::VST : 0); ok && j < nsteps; ++j)
+        ok = mbar_wait_warp(bar(C::B_VEMPTY + j % C::VST), (j / C::VST) & 1, wc, kSiteKVEmpty);
     } else {
       mbar_wait_drain(bar(C::B_QDO), 0, 100000000ull);
-      for (int j = (nsteps > C::STAGES ? nsteps - C::STAGES : 0); j < nsteps; ++j)
-        mbar_wait_drain(bar(C::B_FULL + j % C::STAGES), (j / C::STAGES) & 1, 100000000ull);
+      for (int j = (nk > C::KST ? nk - C::KST : 0); j < nk; ++j)
+        mbar_wait_drain(bar(C::B_KFULL + j % C::KST), (j / C::KST) & 1, 100000000ull);
+      for (int j = (nv > C::VST ? nv - C::VST : 0); j < nv; ++j)
+        mbar_wait_drain(bar(C::B_VFULL + j % C::VST), (j / C::VST) & 1, 100000000ull);
     }
   } else if (warp == C::MMA_WARP) {
     constexpr uint32_t ID_S = idesc_bf16(128, C::BN, false);
     constexpr uint32_t ID_Q = idesc_bf16(128, C::D, true);
-    auto kbuf = [&](int j) { return sbase + C::SMEM_K + (j % C::STAGES) * C::KT_BYTES; };
-    auto vbuf = [&](int j) { return sbase + C::SMEM_V + (j % C::STAGES) * C::KT_BYTES; };
+    auto kbuf = [&](int j) { return sbase + C::SMEM_K + (j % C::KST) * C::KT_BYTES; };
+    auto vbuf = [&](int j) { return sbase + C::SMEM_V + (j % C::VST) * C::KT_BYTES; };
     auto issue_s = [&](int j) -> bool {
-      if (!mbar_wait_warp(bar(C::B_FULL + j % C::STAGES), (j / C::STAGES) & 1, wc, kSiteKFull))
+      if (!mbar_wait_warp(bar(C::B_KFULL + j % C::KST), (j / C::KST) & 1, wc, kSiteKFull))
         return false;
       tc_fence_after();
 #pragma unroll
@@ -599,7 +666,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_commit_elect(bar(C::B_SFULL + j % C::SB));
       return true;
     };
-    auto issue_dp = [&](int j) {
+    auto issue_dp = [&](int j) -> bool {
+      if (!mbar_wait_warp(bar(C::B_VFULL + j % C::VST), (j / C::VST) & 1, wc, kSiteVFull))
+        return false;
+      tc_fence_after();
 #pragma unroll
       for (int kb = 0; kb < C::D / 16; ++kb) {
         const int box = kb / 4, off = (kb % 4) * 32;
@@ -608,24 +678,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       sdesc_sw128(vbuf(j) + box * C::BN * 128 + off, 16, 1024), ID_S, kb > 0);
       }
       tc_commit_elect(bar(C::B_DPFULL + j % C::DB));
+      tc_commit_elect(bar(C::B_VEMPTY + j % C::VST));         // dP(j) is V(j)'s only reader
+      return true;
     };
     // S(j+1) may run ahead of dQ(j): its buffer's last reader, the compute warps'
     // load of S(j+1-SB), happened before they released dS(j+1-SB).  dP(j+1) has to
     // follow dQ(j) unless it has a second buffer.
-    constexpr bool EARLY_S = C::SB == 2 && C::STAGES >= 2;
-    constexpr bool EARLY_DP = EARLY_S && C::DB == 2;
+    constexpr bool EARLY_S = C::SB == 2 && C::KST >= 2;
+    constexpr bool EARLY_DP = EARLY_S && C::DB == 2 && C::VST >= 2;
     bool ok = mbar_wait_warp(bar(C::B_QDO), 0, wc, kSiteQFull);
-    if (ok && nsteps > 0) {
-      ok = issue_s(0);
-      if (ok) issue_dp(0);
-    }
+    if (ok && nsteps > 0) ok = issue_s(0) && issue_dp(0);
     for (int j = 0; j < nsteps && ok; ++j) {
       const int nx = j + 1;
       if (EARLY_S && nx < nsteps) {
         // S(nx) overwrites the buffer S(nx - 2) was loaded from: that load preceded
         // dS(nx - 2), which this warp waited for one iteration ago
         if (!(ok = issue_s(nx))) break;
-        if (EARLY_DP) issue_dp(nx);
+        if (EARLY_DP && !(ok = issue_dp(nx))) break;
       }
       if (!(ok = mbar_wait_warp(bar(C::B_DS + j % C::DB), (j / C::DB) & 1, wc, kSiteDsFull))) break;
       tc_fence_after();
@@ -636,10 +705,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         umma_ts_elect(false, tmem + C::TM_DQ, dpb + half_packed_col<C::BN>(kb),
                       sdesc_sw128(kbuf(j) + kb * 16 * 128, C::BN * 128, 1024), ID_Q,
                       (j > 0 || kb > 0) ? 1u : 0u);
-      tc_commit_elect(bar(C::B_EMPTY + j % C::STAGES));
+      tc_commit_elect(bar(C::B_KEMPTY + j % C::KST));         // S(j) and dQ(j) read K(j)
       if (nx < nsteps) {
         if (!EARLY_S && !(ok = issue_s(nx))) break;
-        if (!EARLY_DP) issue_dp(nx);
+        if (!EARLY_DP && !(ok = issue_dp(nx))) break;
       }
     }
     tc_commit_elect(bar(C::B_ACC));
