@@ -243,11 +243,20 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 }
 
 // Tuning knobs (compile-time): software-exp2 share, pipeline depth, kernel family.
+// software-exp2 share (quarters of the exponentials) per problem class, measured: the
+// two-tile kernel (d = 64, FP8) gains from 2, the split-softmax d = 128 kernel wants 1,
+// the d = 256 kernel (tensor-core bound) none
 #ifndef FA_FWD_EMU
 #define FA_FWD_EMU 1
 #endif
-#ifndef FA_FWD_EMU_MQ
-#define FA_FWD_EMU_MQ FA_FWD_EMU
+#ifndef FA_FWD_D64_EMU
+#define FA_FWD_D64_EMU 2
+#endif
+#ifndef FA_FWD_F8_EMU
+#define FA_FWD_F8_EMU 2
+#endif
+#ifndef FA_FWD_D256_EMU
+#define FA_FWD_D256_EMU 0
 #endif
 #ifndef FA_FWD_WS_INDEP
 #define FA_FWD_WS_INDEP 1
@@ -283,20 +292,20 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #define FA_FWD_F8_KIND 1
 #endif
 
-template <int KIND, int D, bool FP8>
+template <int KIND, int D, bool FP8, int EMU>
 struct FwdPick {
   // stage depths: deep rings where shared memory allows, 2 + 2 for bf16 d = 128
   static constexpr bool kWide = (D == 128 && !FP8);
   static constexpr int KST = kWide ? FA_FWD_D128_KST : 4;
   static constexpr int VST = kWide ? FA_FWD_D128_VST : 4;
   using Cfg = std::conditional_t<
-      KIND == 0, FwdCfg<D, 128, kWide ? 3 : 4, kWide ? 2 : 4, FP8, FA_FWD_EMU>,
+      KIND == 0, FwdCfg<D, 128, kWide ? 3 : 4, kWide ? 2 : 4, FP8, EMU>,
       std::conditional_t<
-          KIND == 1, PPCfg<D, KST, VST, FP8, FA_FWD_EMU, FA_FWD_TAU, FA_FWD_EXPH>,
+          KIND == 1, PPCfg<D, KST, VST, FP8, EMU, FA_FWD_TAU, FA_FWD_EXPH>,
           std::conditional_t<KIND == 2,
-                             WSCfg<D, KST, VST, FP8, FA_FWD_EMU, FA_FWD_EMU_MQ,
+                             WSCfg<D, KST, VST, FP8, EMU, EMU,
                                    FA_FWD_WS_SPLIT != 0, FA_FWD_WS_INDEP != 0>,
-                             SPCfg<D, KST, VST, FP8, FA_FWD_EMU, FA_FWD_SP_SPLIT != 0>>>>;
+                             SPCfg<D, KST, VST, FP8, EMU, FA_FWD_SP_SPLIT != 0>>>>;
   static const char* name() {
     static const std::string n = [] {
       static const char* fam[] = {"fa_fwd_kernel<FwdCfg", "fa_fwd_pp_kernel<PPCfg",
@@ -318,10 +327,10 @@ struct FwdPick {
       return launch_fwd_ws<Cfg>(q, k, v, p, st);
   }
 };
-using FwdD64 = FwdPick<FA_FWD_D64_KIND, 64, false>;
-using FwdD128 = FwdPick<FA_FWD_D128_KIND, 128, false>;
-using FwdF8D128 = FwdPick<FA_FWD_F8_KIND, 128, true>;
-using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_EMU>;
+using FwdD64 = FwdPick<FA_FWD_D64_KIND, 64, false, FA_FWD_D64_EMU>;
+using FwdD128 = FwdPick<FA_FWD_D128_KIND, 128, false, FA_FWD_EMU>;
+using FwdF8D128 = FwdPick<FA_FWD_F8_KIND, 128, true, FA_FWD_F8_EMU>;
+using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_D256_EMU>;
 
 #ifndef FA_BWD_EMU
 #define FA_BWD_EMU 1

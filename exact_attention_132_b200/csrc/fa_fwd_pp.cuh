@@ -319,12 +319,28 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
     const int q_idx = qt * C::BM + row;
     float m = -INFINITY, l = 0.f;
     float qsc = 1.f, vmax = 1.f;
+    // FP8: the V tile scales' max, one load per lane per 32 tiles and a warp reduction;
+    // the per-step K and V scales are fetched a step ahead, so their load latency
+    // overlaps the wait for the scores
+    float ksc_n = 1.f, vsc_n = 1.f;
     if constexpr (C::FP8) {
+      const float* vs = p.v_scale + bh * p.n_st;
       qsc = p.q_scale[bh * p.n_st + qt];
       vmax = 0.f;
-      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[bh * p.n_st + j]);
+      for (int j = threadIdx.x & 31; j < n; j += 32) vmax = fmaxf(vmax, vs[j]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+      ksc_n = p.k_scale[bh * p.n_st];
+      vsc_n = vs[0];
     }
     for (int j = 0; j < n; ++j) {
+      const float ksc = ksc_n, vsc = vsc_n;
+      if constexpr (C::FP8) {
+        if (j + 1 < n) {
+          ksc_n = p.k_scale[bh * p.n_st + j + 1];
+          vsc_n = p.v_scale[bh * p.n_st + j + 1];
+        }
+      }
       if (!(ok = mbar_wait(bar(C::B_SFULL + t), gs & 1, wc, kSiteSFull))) break;
       tc_fence_after();
       float s[C::BN];
@@ -345,8 +361,8 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       }
       float c_j = sl2, fold = 1.f;
       if constexpr (C::FP8) {
-        c_j = sl2 * qsc * p.k_scale[bh * p.n_st + j];
-        fold = 256.f * p.v_scale[bh * p.n_st + j] / vmax;
+        c_j = sl2 * qsc * ksc;
+        fold = 256.f * vsc / vmax;
       }
       // row max: eight independent three-input chains, then a short tree
       float mx[8];
