@@ -262,7 +262,8 @@ def run_ours(args):
 
 
 def run_extras(fa, dev, stream, steps, peak):
-    """fwd+bwd at the two backward workloads and the FP8 forward; device-side seeded inputs."""
+    """fwd+bwd at the two backward workloads, the headline kernel at N=32768 and the FP8
+    forward; device-side seeded inputs."""
     out = {}
     gen = torch.Generator(device=dev)
     for name in ("fwdbwd_d64", "fwdbwd_d256"):
@@ -296,6 +297,23 @@ def run_extras(fa, dev, stream, steps, peak):
                      "ms_fwd_bwd": round(tot / steps, 3), "ms_fwd": round(ftot / steps, 3),
                      "frac_of_bf16_peak": round(fl * steps / (tot * 1e-3) / 1e12 / peak, 4)}
         del q, k, v, do, o, dq, dk, dv, ws
+    # the headline kernel at a long sequence (same kernel, B=1 H=16 N=32768 causal d=128):
+    # context for the per-tile costs that weigh more at N=4096
+    B_, H_, N_, d_ = 1, 16, 32768, 128
+    gen.manual_seed(1002)
+    q, k, v = (torch.randn((B_, H_, N_, d_), generator=gen, device=dev).to(torch.bfloat16)
+               for _ in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty((B_, H_, N_), dtype=torch.float32, device=dev)
+    fl = 4.0 * B_ * H_ * N_ * N_ * d_ / 2
+    n_ = max(3, steps // 2)
+    tot, _ = time_steps(lambda: fa.fa_fwd(q, k, v, o, lse, causal=True, stream=stream), n_, 2,
+                        stream)
+    out["fwd_d128_long"] = {"workload": "bf16 causal forward B=1 H=16 N=32768 d=128 (N(0,1))",
+                            "tflops_fwd": round(fl * n_ / (tot * 1e-3) / 1e12, 2),
+                            "ms_fwd": round(tot / n_, 3),
+                            "frac_of_bf16_peak": round(fl * n_ / (tot * 1e-3) / 1e12 / peak, 4)}
+    del q, k, v, o, lse
     w = workloads.WORKLOADS["fp8_d128"]
     gen.manual_seed(w.seed)
     shp = (w.B, w.H, w.N, w.d)
