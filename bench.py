@@ -215,7 +215,8 @@ def run_ours(args):
 
     extras = {}
     if not args.no_extras:
-        extras = run_extras(fa, dev, stream, max(3, min(args.steps, 10)), peak)
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        extras = run_extras(fa, dev, stream, max(3, min(args.steps, 10)), peak, hbm)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -261,7 +262,7 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def run_extras(fa, dev, stream, steps, peak):
+def run_extras(fa, dev, stream, steps, peak, hbm_peak):
     """fwd+bwd at the two backward workloads, the headline kernel at N=32768 and the FP8
     forward; device-side seeded inputs."""
     out = {}
@@ -314,6 +315,29 @@ def run_extras(fa, dev, stream, steps, peak):
                             "ms_fwd": round(tot / n_, 3),
                             "frac_of_bf16_peak": round(fl * n_ / (tot * 1e-3) / 1e12 / peak, 4)}
     del q, k, v, o, lse
+    # decoding: one query per sequence against a 32k KV cache, 32 query heads on 8 K/V
+    # heads; memory-bound, so reported against the measured HBM bandwidth
+    dw = workloads.DECODE_WORKLOADS["decode_d128"]
+    gen.manual_seed(dw.seed)
+    q = torch.randn((dw.B, dw.Hq, dw.Nq, dw.d), generator=gen, device=dev).to(torch.bfloat16)
+    k, v = (torch.randn((dw.B, dw.Hkv, dw.Nk, dw.d), generator=gen, device=dev).to(torch.bfloat16)
+            for _ in range(2))
+    o = torch.empty_like(q)
+    lse = torch.empty((dw.B, dw.Hq, dw.Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, fa.fa_decode_workspace_size(dw.B, dw.Hq, dw.Hkv, dw.Nq, dw.Nk, dw.d)),
+                     dtype=torch.uint8, device=dev)
+    # the K/V cache (1.07 GB) is far larger than L2, so every launch reads it from HBM
+    tot, _ = time_steps(lambda: fa.fa_decode(q, k, v, o, lse, ws, causal=dw.causal, stream=stream),
+                        steps, 3, stream)
+    gbs = dw.bytes() * steps / (tot * 1e-3) / 1e9
+    out["decode_d128"] = {"workload": f"decode B={dw.B} Hq={dw.Hq} Hkv={dw.Hkv} Nq={dw.Nq} "
+                                      f"Nk={dw.Nk} d={dw.d} causal",
+                          "us_per_call": round(tot / steps * 1e3, 1),
+                          "achieved_gbs": round(gbs, 1),
+                          "hbm_peak_gbs": hbm_peak,
+                          "frac_of_hbm": round(gbs / hbm_peak, 4),
+                          "tflops": round(dw.flops() * steps / (tot * 1e-3) / 1e12, 2)}
+    del q, k, v, o, lse, ws
     w = workloads.WORKLOADS["fp8_d128"]
     gen.manual_seed(w.seed)
     shp = (w.B, w.H, w.N, w.d)

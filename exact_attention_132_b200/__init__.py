@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "FAError", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_size", "fa_last_error_string",
     "fa_get_device_status", "fa_debug_wait_timeout_selftest", "fa_version", "fa_fwd_kernel_name",
-    "attention_forward",
+    "fa_decode", "fa_decode_workspace_size", "attention_forward", "attention_decode",
     "attention_forward_fp8", "attention_backward", "LIB_PATH", "lib",
 ]
 
@@ -53,6 +53,10 @@ def _load() -> ctypes.CDLL:
     L.fa_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     L.fa_debug_wait_timeout_selftest.argtypes = [i, vp]
     L.fa_version.argtypes = []
+    L.fa_decode_workspace_size.argtypes = [i, i, i, i, i, i]
+    L.fa_decode_workspace_size.restype = sz
+    L.fa_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
+    L.fa_decode.restype = ctypes.c_int
     L.fa_fwd_kernel_name.argtypes = [i, i]
     L.fa_fwd_kernel_name.restype = ctypes.c_char_p
     for name in ("fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_get_device_status",
@@ -224,3 +228,40 @@ def attention_backward(q, k, v, o, dO, lse, causal: bool = False, scale: float |
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
     fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, scale=scale, causal=causal)
     return dq, dk, dv
+
+
+# ------------------------------------------------------------------ decoding (GQA / MQA)
+def fa_decode_workspace_size(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int) -> int:
+    return int(lib.fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d))
+
+
+def fa_decode(q, k, v, o, lse, workspace, scale: float | None = None, causal: bool = False,
+              stream=None):
+    """Few queries ([B, Hq, Nq, d]) against long K/V ([B, Hkv, Nk, d]); causal queries sit
+    at the end of the sequence.  Writes o (bf16) and lse (fp32 [B, Hq, Nq], or None)."""
+    B, Hq, Nq, d = _bhnd(q, "q", torch.bfloat16)
+    Bk, Hkv, Nk, dk = _bhnd(k, "k", torch.bfloat16)
+    if (Bk, dk) != (B, d) or tuple(v.shape) != tuple(k.shape) or v.dtype != torch.bfloat16:
+        raise ValueError("k and v must be bf16 [B, Hkv, Nk, d] with q's B and d")
+    if not v.is_contiguous():
+        raise ValueError("v must be contiguous")
+    if _bhnd(o, "o", torch.bfloat16) != (B, Hq, Nq, d):
+        raise ValueError("o shape differs from q")
+    if lse is not None and (tuple(lse.shape) != (B, Hq, Nq) or lse.dtype != torch.float32):
+        raise ValueError("lse must be fp32 [B, Hq, Nq]")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.fa_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, sc,
+                         1 if causal else 0, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def attention_decode(q, k, v, causal: bool = False, scale: float | None = None):
+    """Allocate O, LSE and the workspace with torch and run fa_decode; returns (o, lse)."""
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    nbytes = fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    fa_decode(q, k, v, o, lse, ws, scale=scale, causal=causal)
+    return o, lse

@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfa.so")
 SOURCES = ["fa_api.cu"]
-HEADERS = ["sm100_ptx.cuh", "fa_fwd.cuh", "fa_fwd_pp.cuh", "fa_fwd_ws.cuh", "fa_fwd_sp.cuh", "fa_bwd.cuh"]
+HEADERS = ["sm100_ptx.cuh", "fa_fwd.cuh", "fa_fwd_pp.cuh", "fa_fwd_ws.cuh", "fa_fwd_sp.cuh", "fa_decode.cuh", "fa_bwd.cuh"]
 
 
 def nvcc_path() -> str:

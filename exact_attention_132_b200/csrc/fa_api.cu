@@ -18,6 +18,7 @@
 #include "fa_fwd_pp.cuh"
 #include "fa_fwd_ws.cuh"
 #include "fa_fwd_sp.cuh"
+#include "fa_decode.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa {
@@ -453,6 +454,83 @@ fa_status noalloc_scratch(float** out) {
   return FA_OK;
 }
 
+// ---------------------------------------------------------------- decoding
+using DecD64 = DecCfg<64, 6, 6>;
+using DecD128 = DecCfg<128, 3, 3>;
+using DecD256 = DecCfg<256, 2, 2>;
+
+struct DecPlan {
+  int BHkv, R, bn, n_kt, split_tiles, n_split;
+  size_t part_o_bytes, part_lse_bytes, total;
+};
+
+fa_status dec_check(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                    bool* empty) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0)
+    return fail(FA_ERR_INVALID_ARG, "negative size B=%d Hq=%d Hkv=%d Nq=%d Nk=%d", B, Hq, Hkv, Nq, Nk);
+  if (!std::isfinite(scale) || !(scale > 0.f))
+    return fail(FA_ERR_INVALID_ARG, "scale must be finite and > 0 (got %g)", static_cast<double>(scale));
+  if (d != 64 && d != 128 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
+  *empty = (B == 0 || Hq == 0 || Nq == 0);
+  if (*empty) return FA_OK;
+  if (Hkv == 0 || Hq % Hkv != 0)
+    return fail(FA_ERR_INVALID_ARG, "Hq=%d must be a multiple of Hkv=%d", Hq, Hkv);
+  if (static_cast<long long>(Hq / Hkv) * Nq > 128)
+    return fail(FA_ERR_INVALID_ARG, "(Hq/Hkv)*Nq = %lld query rows per key/value head exceed 128",
+                static_cast<long long>(Hq / Hkv) * Nq);
+  if (Nk < 1) return fail(FA_ERR_INVALID_ARG, "Nk must be >= 1");
+  if (causal && Nq > Nk) return fail(FA_ERR_INVALID_ARG, "causal decoding needs Nq <= Nk");
+  if (static_cast<long long>(B) * Hkv > (1ll << 30)) return fail(FA_ERR_INVALID_ARG, "B*Hkv too large");
+  return FA_OK;
+}
+
+// Split count: about two work items per SM, at least one key tile per split.
+fa_status dec_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, DecPlan* pl) {
+  DeviceInfo* di = nullptr;
+  if (fa_status s = device_info(&di)) return s;
+  pl->BHkv = B * Hkv;
+  pl->R = (Hq / Hkv) * Nq;
+  pl->bn = d <= 128 ? 128 : 64;
+  pl->n_kt = (Nk + pl->bn - 1) / pl->bn;
+  const long long target = 2ll * di->sms;
+  long long ns = (target + pl->BHkv - 1) / pl->BHkv;
+  if (ns < 1) ns = 1;
+  if (ns > pl->n_kt) ns = pl->n_kt;
+  pl->split_tiles = static_cast<int>((pl->n_kt + ns - 1) / ns);
+  pl->n_split = (pl->n_kt + pl->split_tiles - 1) / pl->split_tiles;
+  const size_t rows = static_cast<size_t>(pl->BHkv) * pl->n_split * pl->R;
+  pl->part_o_bytes = (rows * d * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  pl->part_lse_bytes = (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  pl->total = pl->part_o_bytes + pl->part_lse_bytes;
+  return FA_OK;
+}
+
+template <class C>
+fa_status launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, DecParams p,
+                        cudaStream_t stream) {
+  DeviceInfo* di = nullptr;
+  if (fa_status s = device_info(&di)) return s;
+  CUtensorMap mq, mk, mv;
+  if (fa_status s = make_map(&mq, q, false, C::D, p.R, p.BHkv, C::BM)) return s;
+  if (fa_status s = make_map(&mk, k, false, C::D, p.Nk, p.BHkv, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, false, C::D, p.Nk, p.BHkv, C::BN)) return s;
+  auto kern = fa_decode_split_kernel<C>;
+  if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
+  p.status = di->status;
+  p.timeout_ns = kWaitTimeoutNs;
+  const int grid = p.total_items < di->sms ? p.total_items : di->sms;
+  kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode split kernel launch");
+  const long long warps = static_cast<long long>(p.BHkv) * p.R;
+  const long long blocks = (warps * 32 + 255) / 256;
+  fa_decode_combine_kernel<C::D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, o, lse);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode combine kernel launch");
+  return FA_OK;
+}
+
 }  // namespace fa
 
 using namespace fa;
@@ -620,6 +698,49 @@ fa_status fa_debug_wait_timeout_selftest(int timeout_us, void* stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
   return FA_OK;
+}
+
+size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  bool empty = false;
+  if (dec_check(B, Hq, Hkv, Nq, Nk, d, 1.f, 0, &empty) != FA_OK || empty) return 0;
+  DecPlan pl;
+  if (dec_plan(B, Hq, Hkv, Nq, Nk, d, &pl) != FA_OK) return 0;
+  return pl.total;
+}
+
+fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  bool empty = false;
+  if (fa_status s = dec_check(B, Hq, Hkv, Nq, Nk, d, scale, causal, &empty)) return s;
+  if (empty) return FA_OK;
+  const void* ptrs[] = {q, k, v, o, workspace};
+  const char* names[] = {"q", "k", "v", "o", "workspace"};
+  if (fa_status s = check_ptrs(ptrs, names, 5)) return s;
+  if (lse && !aligned16(lse)) return fail(FA_ERR_INVALID_ARG, "lse is not 16-byte aligned");
+  DecPlan pl;
+  if (fa_status s = dec_plan(B, Hq, Hkv, Nq, Nk, d, &pl)) return s;
+  if (workspace_bytes < pl.total)
+    return fail(FA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, pl.total);
+  DecParams p{};
+  p.BHkv = pl.BHkv;
+  p.R = pl.R;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.causal = causal ? 1 : 0;
+  p.n_kt = pl.n_kt;
+  p.split_tiles = pl.split_tiles;
+  p.n_split = pl.n_split;
+  p.total_items = pl.BHkv * pl.n_split;
+  p.scale = scale;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.part_o_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_decode<DecD64>(q, k, v, o, lse, p, st);
+    case 128: return launch_decode<DecD128>(q, k, v, o, lse, p, st);
+    default: return launch_decode<DecD256>(q, k, v, o, lse, p, st);
+  }
 }
 
 int fa_version(void) { return 100; }

@@ -148,6 +148,42 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          const void* dO, const float* lse, void* dq, void* dk, void* dv,
                          int B, int H, int N, int d, float scale, int causal, void* stream);
 
+/*
+ * Decoding: few query rows against a long key/value sequence, with grouped query
+ * heads (GQA / MQA).  Same exact attention as fa_fwd.  Decoding reads Q of length 1
+ * against the whole KV cache, so reading K and V bounds it ("FlashAttentionとは？…"
+ * (issoh.co.jp), section 短い系列の効果とデコード向け最適化の違い); shared K/V heads
+ * are the GQA/MQA of "FlashAttention — フラッシュアテンション" (systems-analysis.info),
+ * section FlashAttention-2（2023年）.  The key split and its merge are the
+ * online-softmax rescale applied across key ranges:
+ *   O[b,h,i,:] = softmax_j(scale * q[b,h,i,:] . k[b,h/g,j,:]) v[b,h/g,j,:],
+ *   g = Hq / Hkv, causal: query i sees keys j <= Nk - Nq + i (the queries are the
+ *   last Nq positions of the sequence).
+ *
+ * fa_decode_workspace_size — bytes of device workspace fa_decode needs (partial
+ * results of the key splits; the split count follows the current device's SM
+ * count).  0 for arguments fa_decode would reject.
+ */
+size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+
+/*
+ * fa_decode — O and row logsumexp for the layout above.
+ *   q          bf16 [B, Hq, Nq, d], d contiguous       (device, read)
+ *   k, v       bf16 [B, Hkv, Nk, d]                    (device, read)
+ *   o          bf16 [B, Hq, Nq, d]                     (device, written)
+ *   lse        fp32 [B, Hq, Nq] natural-log logsumexp  (device, written; may be NULL)
+ *   d in {64, 128, 256}; Hq % Hkv == 0; (Hq / Hkv) * Nq <= 128; 1 <= Nq; 1 <= Nk;
+ *   causal requires Nq <= Nk.
+ *   workspace  >= fa_decode_workspace_size() bytes of device memory, 16-byte aligned,
+ *              owned by the caller, contents ignored and overwritten.
+ * Asynchronous on `stream`; allocates nothing.  Errors: FA_ERR_INVALID_ARG for a
+ * null or misaligned pointer, out-of-range sizes or a too-small workspace (nothing
+ * launched); FA_ERR_UNSUPPORTED for another d; FA_ERR_CUDA if a launch fails.
+ */
+fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* fa_last_error_string — text of the calling thread's last failure ("" if none). */
 const char* fa_last_error_string(void);
 

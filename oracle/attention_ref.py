@@ -248,3 +248,39 @@ def attention_bwd_rows_dq(q, k, v, do, scale: float, causal: bool, picks):
         D = (p * dp).sum(axis=1, keepdims=True)
         out[n] = (scale * ((p * (dp - D)) @ k2))[0]
     return out
+
+
+def attention_decode(q, k, v, scale: float, causal: bool):
+    """Few queries against a long key/value sequence with grouped heads, by definition.
+
+    q [B, Hq, Nq, d]; k, v [B, Hkv, Nk, d] with Hq = g * Hkv; query head h reads
+    key/value head h // g (the GQA / MQA sharing of "FlashAttention —
+    フラッシュアテンション" (systems-analysis.info), section FlashAttention-2（2023年）).
+    Causal reading: the Nq queries are the last Nq positions of the Nk-long sequence
+    (decoding with a KV cache, "FlashAttentionとは？…" (issoh.co.jp), section
+    短い系列の効果とデコード向け最適化の違い), so query i sees keys j <= Nk - Nq + i; for
+    Nq == Nk this is the lower-triangular mask of attention_fwd.
+    Returns (O [B, Hq, Nq, d], LSE [B, Hq, Nq]) in fp64: the full Nq x Nk score
+    matrix, two-pass softmax, O = P V, LSE = m + ln(sum exp(S - m)).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    g = Hq // Hkv
+    O = np.empty((B, Hq, Nq, v.shape[3]))
+    L = np.empty((B, Hq, Nq))
+    last = np.arange(Nq)[:, None] + (Nk - Nq)          # last visible key of each query
+    cols = np.arange(Nk)[None, :]
+    for b in range(B):
+        for h in range(Hq):
+            s = (q[b, h] @ k[b, h // g].T) * scale
+            if causal:
+                s = np.where(cols > last, -np.inf, s)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            l = e.sum(axis=1, keepdims=True)
+            O[b, h] = (e / l) @ v[b, h // g]
+            L[b, h] = (m + np.log(l))[:, 0]
+    return O, L

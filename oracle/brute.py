@@ -55,3 +55,30 @@ def brute_bwd(q, k, v, do, scale: float, causal: bool):
     dQ = [[scale * sum(dS[i][j] * k[j][c] for j in range(Nk)) for c in range(d)] for i in range(N)]
     dK = [[scale * sum(dS[i][j] * q[i][c] for i in range(N)) for c in range(d)] for j in range(Nk)]
     return dQ, dK, dV
+
+
+def brute_decode(q, k, v, scale: float, causal: bool):
+    """One query head against its key/value head, queries at the END of the sequence.
+
+    q: [Nq][d], k, v: [Nk][d] nested lists.  Query i sits at position Nk - Nq + i, so
+    with causal it sees keys j <= Nk - Nq + i.  Returns (O [Nq][dv], LSE [Nq]).
+    """
+    Nq, Nk, dv = len(q), len(k), len(v[0])
+    O, LSE = [], []
+    for i in range(Nq):
+        pos = Nk - Nq + i
+        s = []
+        for j in range(Nk):
+            if causal and j > pos:
+                s.append(None)
+                continue
+            acc = 0.0
+            for c in range(len(q[i])):
+                acc += q[i][c] * k[j][c]
+            s.append(acc * scale)
+        m = max(x for x in s if x is not None)
+        e = [0.0 if x is None else math.exp(x - m) for x in s]
+        den = sum(e)
+        O.append([sum(e[j] / den * v[j][c] for j in range(Nk)) for c in range(dv)])
+        LSE.append(m + math.log(den))
+    return O, LSE

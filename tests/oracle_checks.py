@@ -246,3 +246,102 @@ def check_torch_autograd_bwd(bwd, N=17, d=8) -> bool:
 
 
 BWD_CHECKS = [check_golden_tiny_bwd, check_brute_bwd, check_bwd_invariants, check_torch_autograd_bwd]
+
+
+# --------------------------------------------------------------------------- decoding checks
+# decode signature: dec(q [B,Hq,Nq,d], k [B,Hkv,Nk,d], v, scale, causal) -> (O, LSE)
+def _dec_inputs(seed, B=1, Hq=4, Hkv=2, Nq=3, Nk=7, d=4, dv=None):
+    r = _rng(seed)
+    q = r.standard_normal((B, Hq, Nq, d))
+    k = r.standard_normal((B, Hkv, Nk, d))
+    v = r.standard_normal((B, Hkv, Nk, dv or d))
+    return q, k, v
+
+
+def check_dec_brute(dec) -> bool:
+    """Scalar brute force per query head, key/value head h // g, queries at the end."""
+    from oracle import brute_decode
+    ok = True
+    for (Hq, Hkv, Nq, Nk) in ((4, 2, 3, 7), (3, 1, 2, 5), (2, 2, 4, 4)):
+        q, k, v = _dec_inputs(23 + Nk, Hq=Hq, Hkv=Hkv, Nq=Nq, Nk=Nk)
+        for causal in (False, True):
+            o, lse = dec(q, k, v, 0.41, causal)
+            for h in range(Hq):
+                bo, bl = brute_decode(q[0, h].tolist(), k[0, h // (Hq // Hkv)].tolist(),
+                                      v[0, h // (Hq // Hkv)].tolist(), 0.41, causal)
+                ok &= _close(o[0, h], bo, 1e-12) and _close(lse[0, h], bl, 1e-12)
+    return ok
+
+
+def check_dec_q_zero(dec, Nq=5, Nk=23) -> bool:
+    """Q = 0: query i averages the keys it sees, Nk - Nq + i + 1 of them when causal."""
+    q, k, v = _dec_inputs(29, Hq=4, Hkv=2, Nq=Nq, Nk=Nk, d=3)
+    q[:] = 0.0
+    ok = True
+    for causal in (False, True):
+        o, lse = dec(q, k, v, 0.7, causal)
+        for h in range(4):
+            vv = v[0, h // 2]
+            for i in range(Nq):
+                cnt = (Nk - Nq + i + 1) if causal else Nk
+                ok &= _close(o[0, h, i], vv[:cnt].mean(axis=0), 1e-12)
+                ok &= abs(lse[0, h, i] - math.log(cnt)) < 1e-12
+    return ok
+
+
+def check_dec_constant_v(dec) -> bool:
+    """Every value row equal to c gives O = c for every query (weights sum to one)."""
+    q, k, v = _dec_inputs(31, Nq=4, Nk=9)
+    v[:] = np.array([0.5, -1.25, 2.0, 3.5])
+    o, _ = dec(q, k, v, 0.9, True)
+    return _close(o, np.broadcast_to(np.array([0.5, -1.25, 2.0, 3.5]), o.shape), 1e-12)
+
+
+def check_dec_torch_sdpa(dec) -> bool:
+    """fp64 torch SDPA with the key/value heads repeated per group and an explicit
+    end-aligned causal mask (query i sees keys j <= Nk - Nq + i)."""
+    q, k, v = _dec_inputs(37, B=2, Hq=6, Hkv=3, Nq=5, Nk=13, d=8)
+    ok = True
+    for causal in (False, True):
+        tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+        tk, tv = tk.repeat_interleave(2, dim=1), tv.repeat_interleave(2, dim=1)
+        mask = None
+        if causal:
+            i = torch.arange(5)[:, None]
+            j = torch.arange(13)[None, :]
+            mask = j <= i + (13 - 5)
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask,
+                                                               scale=0.33).numpy()
+        s = (tq @ tk.transpose(-1, -2)) * 0.33
+        if causal:
+            s = s.masked_fill(~mask, float("-inf"))
+        lref = torch.logsumexp(s, dim=-1).numpy()
+        o, lse = dec(q, k, v, 0.33, causal)
+        ok &= _close(o, ref, 1e-12) and _close(lse, lref, 1e-12)
+    return ok
+
+
+def check_dec_square_is_forward(dec) -> bool:
+    """Nq == Nk with one query head per key/value head is the ordinary forward: the
+    end-aligned mask becomes the lower triangle (brute_fwd, the forward's own pin)."""
+    q, k, v = _dec_inputs(41, Hq=2, Hkv=2, Nq=6, Nk=6)
+    ok = True
+    for causal in (False, True):
+        o, lse = dec(q, k, v, 0.5, causal)
+        for h in range(2):
+            bo, bl = brute_fwd(q[0, h].tolist(), k[0, h].tolist(), v[0, h].tolist(), 0.5, causal)
+            ok &= _close(o[0, h], bo, 1e-12) and _close(lse[0, h], bl, 1e-12)
+    return ok
+
+
+def check_dec_last_query_sees_all(dec) -> bool:
+    """The last query (position Nk - 1) sees every key: causal == non-causal for it."""
+    q, k, v = _dec_inputs(43, Nq=3, Nk=11)
+    oc_, lc = dec(q, k, v, 0.6, True)
+    on, ln = dec(q, k, v, 0.6, False)
+    return _close(oc_[:, :, -1], on[:, :, -1], 1e-13) and _close(lc[:, :, -1], ln[:, :, -1], 1e-13) \
+        and not _close(oc_[:, :, 0], on[:, :, 0], 1e-6)
+
+
+DEC_CHECKS = [check_dec_brute, check_dec_q_zero, check_dec_constant_v, check_dec_torch_sdpa,
+              check_dec_square_is_forward, check_dec_last_query_sees_all]

@@ -99,3 +99,22 @@ def test_python_wrappers_validate_shapes():
         fa.fa_fwd(q, q[:, :1], q, q)
     with pytest.raises(ValueError):
         fa.fa_fwd(q, q, q, q)   # CPU tensors are rejected: no CPU path exists
+
+
+def _dec(q=1, k=1, v=1, o=1, lse=None, B=1, Hq=8, Hkv=2, Nq=1, Nk=300, d=128, scale=0.1,
+         causal=0, ws=1, ws_bytes=1 << 30):
+    P = lambda x: None if x is None else ctypes.c_void_p(16 * x)
+    return fa.lib.fa_decode(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                            P(ws), ws_bytes, None)
+
+
+def test_decode_argument_errors_return_before_any_cuda_call():
+    assert _dec(d=96) == 2                              # unsupported head dim
+    assert _dec(Hq=6, Hkv=4) == 1                       # Hq not a multiple of Hkv
+    assert _dec(Hq=64, Hkv=1, Nq=4) == 1                # 256 rows per key/value head
+    assert _dec(Nk=0) == 1
+    assert _dec(causal=1, Nq=4, Nk=3) == 1              # causal needs Nq <= Nk
+    assert _dec(scale=float("nan")) == 1
+    assert _dec(B=-1) == 1
+    assert _dec(Nq=0) == 0 and _dec(B=0) == 0           # empty problems are no-ops
+    assert fa.fa_decode_workspace_size(1, 6, 4, 1, 100, 128) == 0

@@ -111,3 +111,61 @@ def test_backward_mutant_is_caught(name):
         if not ok:
             failures.append(chk.__name__)
     assert failures, f"mutant {name} passed every backward check"
+
+
+# ----------------------------------------------------------------------------- decoding
+def _dec_generic(q, k, v, scale, causal, *, head_mod=False, offset=0, top_left=False,
+                 use_scale=True, lse_no_max=False):
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    B, Hq, Nq, _ = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    O = np.empty((B, Hq, Nq, v.shape[3]))
+    L = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            kh = h % Hkv if head_mod else h // g
+            s = q[b, h] @ k[b, kh].T
+            if use_scale:
+                s = s * scale
+            if causal:
+                i = np.arange(Nq)[:, None]
+                j = np.arange(Nk)[None, :]
+                last = i if top_left else i + (Nk - Nq) + offset
+                s = np.where(j > last, -np.inf, s)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            l = e.sum(axis=1, keepdims=True)
+            O[b, h] = (e / l) @ v[b, kh]
+            L[b, h] = (np.log(l) if lse_no_max else m + np.log(l))[:, 0]
+    return O, L
+
+
+MUTANTS_DEC = {
+    "kv_head_modulo": dict(head_mod=True),
+    "mask_from_start": dict(top_left=True),
+    "mask_one_key_short": dict(offset=-1),
+    "mask_one_key_long": dict(offset=1),
+    "dropped_scale": dict(use_scale=False),
+    "lse_without_max": dict(lse_no_max=True),
+}
+
+
+def test_unmutated_decode_passes():
+    for chk in oc.DEC_CHECKS:
+        assert chk(_dec_generic), chk.__name__
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS_DEC))
+def test_decode_mutant_is_caught(name):
+    kw = MUTANTS_DEC[name]
+    f = lambda q, k, v, s, c: _dec_generic(q, k, v, s, c, **kw)
+    failures = []
+    for chk in oc.DEC_CHECKS:
+        try:
+            ok = chk(f)
+        except Exception:
+            ok = False
+        if not ok:
+            failures.append(chk.__name__)
+    assert failures, f"mutant {name} passed every decoding check"

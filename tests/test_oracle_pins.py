@@ -83,3 +83,8 @@ def test_row_blocking_is_exact(monkeypatch):
     assert np.abs(o1 - o2).max() < 1e-14 and np.abs(l1 - l2).max() < 1e-14
     for a, b in zip(g1, g2):
         assert np.abs(a - b).max() < 1e-13
+
+
+@pytest.mark.parametrize("check", oc.DEC_CHECKS, ids=lambda f: f.__name__)
+def test_oracle_decode_pins(check):
+    assert check(oracle.attention_decode)

@@ -164,3 +164,49 @@ def make_small(B: int, H: int, N: int, d: int, causal: bool, seed: int = 7, std:
     """An ad-hoc small workload for parity tests (several tiles plus a ragged tail)."""
     return Workload(f"small_b{B}h{H}n{N}d{d}{'c' if causal else ''}", B, H, N, d, causal,
                     backward=backward, std=std, seed=seed, scale=scale)
+
+
+# ----------------------------------------------------------------------------- decoding
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Few queries against a long key/value sequence with grouped heads."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed: int
+    std: float = 1.0
+
+    @property
+    def sm_scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        """4 * B * Hq * Nq * Nk * d (every query sees almost every key; the end-aligned
+        causal mask hides at most Nq - 1 keys)."""
+        return 4.0 * self.B * self.Hq * self.Nq * self.Nk * self.d
+
+    def bytes(self) -> int:
+        """Algorithmic HBM bytes: Q, K, V read and O written in bf16, LSE in fp32."""
+        return 2 * (self.B * self.Hq * self.Nq * self.d * 2 + self.B * self.Hkv * self.Nk * self.d * 2) \
+            + 4 * self.B * self.Hq * self.Nq
+
+
+DECODE_WORKLOADS = {
+    # one new token per sequence, 32 query heads sharing 8 key/value heads, 32k cache
+    "decode_d128": DecodeWorkload("decode_d128", 8, 32, 8, 1, 32768, 128, True, seed=1006),
+}
+
+
+def make_decode_inputs(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, seed: int,
+                       std: float = 1.0):
+    """CPU bf16 q [B, Hq, Nq, d], k, v [B, Hkv, Nk, d], N(0, std^2), one seeded generator."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    q = _randn(gen, (B, Hq, Nq, d), std).to(torch.bfloat16)
+    k = _randn(gen, (B, Hkv, Nk, d), std).to(torch.bfloat16)
+    v = _randn(gen, (B, Hkv, Nk, d), std).to(torch.bfloat16)
+    return q, k, v
