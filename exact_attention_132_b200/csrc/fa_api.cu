@@ -274,6 +274,9 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #ifndef FA_FWD_D128_VST
 #define FA_FWD_D128_VST 2
 #endif
+#ifndef FA_FWD_WS_TAU
+#define FA_FWD_WS_TAU 8
+#endif
 #ifndef FA_FWD_TAU
 #define FA_FWD_TAU 0
 #endif
@@ -305,7 +308,7 @@ struct FwdPick {
           KIND == 1, PPCfg<D, KST, VST, FP8, EMU, FA_FWD_TAU, FA_FWD_EXPH>,
           std::conditional_t<KIND == 2,
                              WSCfg<D, KST, VST, FP8, EMU, EMU,
-                                   FA_FWD_WS_SPLIT != 0, FA_FWD_WS_INDEP != 0>,
+                                   FA_FWD_WS_SPLIT != 0, FA_FWD_WS_INDEP != 0, FA_FWD_WS_TAU>,
                              SPCfg<D, KST, VST, FP8, EMU, FA_FWD_SP_SPLIT != 0>>>>;
   static const char* name() {
     static const std::string n = [] {

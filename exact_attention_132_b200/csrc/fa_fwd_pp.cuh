@@ -35,7 +35,8 @@ struct PPCfg {
   // rescaled) only when a row max exceeds it by more than TAU (log2 units), so
   // P <= 2^TAU.  With TAU > 0 the row sum l adds the bf16-ROUNDED probabilities, the
   // very values the P V product uses, so O = sum P V / sum P is a convex combination
-  // whose weights carry no bias from rounding the largest probability.
+  // whose weights carry no bias from rounding the largest probability; the logsumexp
+  // uses a second, unrounded sum.
   static constexpr float TAU = FP8 ? 0.f : static_cast<float>(TAU_);
   // bf16 only: exponentials on the special-function unit in half precision, two
   // values per instruction (ex2.approx.f16x2).
@@ -317,7 +318,8 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
     const int n = pp_kv_tiles<C>(p, qt);
     if (n == 0) continue;
     const int q_idx = qt * C::BM + row;
-    float m = -INFINITY, l = 0.f;
+    constexpr bool kFusedSum = !C::FP8 && (C::TAU > 0.f || C::EXPH);
+    float m = -INFINITY, l = 0.f, lx = 0.f;   // lx: unrounded row sum (fused path)
     float qsc = 1.f, vmax = 1.f;
     // FP8: the V tile scales' max, one load per lane per 32 tiles and a warp reduction;
     // the per-step K and V scales are fetched a step ahead, so their load latency
@@ -381,6 +383,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       const uint64_t c2 = f2_pack(c_j, c_j);
       const uint64_t nm2 = f2_pack(-m_use, -m_use);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint64_t accx[4] = {0ull, 0ull, 0ull, 0ull};   // unrounded sums, fused path
       // bf16 with TAU > 0 or half-precision exponentials: exponentials, rounding to
       // bf16 and the row sum of the rounded values in one pass
       uint32_t pk[C::BN / 2];
@@ -405,6 +408,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
           pk[c / 2] = u;
           acc[(c / 2) % 4] = f2_add(acc[(c / 2) % 4],
                                     f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
+          accx[(c / 2) % 4] = f2_add(accx[(c / 2) % 4], p2);
         }
       };
       auto exps = [&](auto emu_tag) {
@@ -439,6 +443,11 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
       l = l * alpha + (sa + sb);
+      if constexpr (kFused) {
+        float xa, xb;
+        f2_unpack(f2_add(f2_add(accx[0], accx[1]), f2_add(accx[2], accx[3])), xa, xb);
+        lx = lx * alpha + (xa + xb);
+      }
       if constexpr (kFused) {
 #pragma unroll
         for (int c = 0; c < C::BN / 2; c += 32) {
@@ -518,7 +527,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       }
     }
     if (row_ok && p.lse != nullptr)
-      p.lse[static_cast<size_t>(bh) * p.N + q_idx] = (m + __log2f(l)) * LN2;
+      p.lse[static_cast<size_t>(bh) * p.N + q_idx] = (m + __log2f(kFusedSum ? lx : l)) * LN2;
     tc_fence_before();
   }
 }

@@ -28,7 +28,7 @@
 namespace fa {
 
 template <int D_, int KST_, int VST_, bool FP8_, int EMU_ = 1, int EMU_MQ_ = EMU_, bool SPLIT_ = false,
-          bool INDEP_ = false>
+          bool INDEP_ = false, int TAU_ = 0>
 struct WSCfg {
   static constexpr int D = D_;
   static constexpr int BN = 128;
@@ -46,6 +46,12 @@ struct WSCfg {
   // row never wait for each other inside the key loop; they are combined once per tile.
   static constexpr bool INDEP = INDEP_;
   static constexpr bool SEPARATE_P = false;
+  // bf16, independent halves only: a row's reference max moves (and O_h is rescaled)
+  // only when the row max exceeds it by more than TAU (log2 units), so P <= 2^TAU.  O is
+  // then normalised by the sum of the bf16-ROUNDED probabilities, the very values the
+  // P V product uses, so the largest probability (no longer exactly 1) carries no
+  // rounding bias into O; the logsumexp uses the unrounded sum.
+  static constexpr float TAU = FP8 ? 0.f : static_cast<float>(TAU_);
   static constexpr int HALF = BN / 2;                 // score columns per softmax warp
   static constexpr int DH = D / 2;                    // output columns per softmax warp
   static constexpr int ELEM = FP8 ? 1 : 2;
@@ -683,7 +689,7 @@ __device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tme
     fwd_decode_item(p, w, bh, qt);
     const int n = fwd_num_kv_tiles<C>(p, qt);
     const int q_idx = qt * C::BM + row;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f, lx = 0.f;   // lx: unrounded row sum (TAU > 0)
     float qsc = 1.f, vmax = 1.f;
     if constexpr (C::FP8) {
       qsc = p.q_scale[bh * p.n_st + qt];
@@ -727,13 +733,16 @@ __device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tme
 #pragma unroll
         for (int i = 0; i < 4; ++i) mx[i] = max3f(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
       const float m_cand = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c_j;
-      const bool raise = m_cand > m;
+      const bool raise = m_cand > m + C::TAU;
       const float m_new = raise ? m_cand : m;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = raise ? ex2(m - m_use) : 1.f;
       const uint64_t c2 = f2_pack(c_j, c_j);
       const uint64_t nm2 = f2_pack(-m_use, -m_use);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint64_t accr[4] = {0ull, 0ull, 0ull, 0ull};    // sums of the rounded P (TAU > 0)
+      constexpr bool kRounded = C::TAU > 0.f;
+      uint32_t pk[kRounded ? C::HALF / 2 : 1];
       auto exps = [&](auto emu_tag) {
         constexpr int kEmu = decltype(emu_tag)::value;
 #pragma unroll
@@ -748,7 +757,16 @@ __device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tme
             p2 = f2_pack(ex2(xa), ex2(xb));
           }
           acc[(c / 2) % 4] = f2_add(acc[(c / 2) % 4], p2);
-          f2_unpack(p2, s[c], s[c + 1]);
+          if constexpr (kRounded) {
+            float pa, pb;
+            f2_unpack(p2, pa, pb);
+            const uint32_t u = pack_bf16x2(pa, pb);
+            pk[c / 2] = u;
+            accr[(c / 2) % 4] = f2_add(accr[(c / 2) % 4], f2_pack(__uint_as_float(u << 16),
+                                                                   __uint_as_float(u & 0xFFFF0000u)));
+          } else {
+            f2_unpack(p2, s[c], s[c + 1]);
+          }
         }
       };
       if (need_mask)
@@ -759,9 +777,18 @@ __device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tme
         exps(std::integral_constant<int, C::EMU>{});
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
-      l = l * alpha + (sa + sb);
+      if constexpr (kRounded) {
+        float ra, rb;
+        f2_unpack(f2_add(f2_add(accr[0], accr[1]), f2_add(accr[2], accr[3])), ra, rb);
+        l = l * alpha + (ra + rb);
+        lx = lx * alpha + (sa + sb);
+      } else {
+        l = l * alpha + (sa + sb);
+      }
       // P_h(j) over this half's own score columns
-      if constexpr (C::FP8) {
+      if constexpr (kRounded) {
+        tmem_st32(s_cols, *reinterpret_cast<uint32_t(*)[32]>(pk));
+      } else if constexpr (C::FP8) {
         uint32_t r[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -793,6 +820,7 @@ __device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tme
     // combine the halves: O = sum_h O_h 2^(m_h - m), l = sum_h l_h 2^(m_h - m)
     xbuf[half * 128 + row] = m;
     xbuf[(2 + half) * 128 + row] = l;
+    if constexpr (C::TAU > 0.f) xbuf[(4 + half) * 128 + row] = lx;
     mbar_arrive_warp(b_x);
     if (!mbar_wait(b_x, xc & 1, wc, kSiteXchg)) { ok = false; break; }
     ++xc;
@@ -803,6 +831,9 @@ __device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tme
     const float e_me = ex2(((m == -INFINITY) ? m_ref : m) - m_ref) * (m == -INFINITY ? 0.f : 1.f);
     const float e_ot = ex2(((m_o == -INFINITY) ? m_ref : m_o) - m_ref) * (m_o == -INFINITY ? 0.f : 1.f);
     const float l_row = l * e_me + l_o * e_ot;
+    // the logsumexp from the unrounded sums (TAU > 0) or the one sum kept
+    float lx_row = l_row;
+    if constexpr (C::TAU > 0.f) lx_row = lx * e_me + xbuf[(4 + (half ^ 1)) * 128 + row] * e_ot;
     const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / l_row;
     const float w_self = e_me * inv_l, w_other = e_ot * inv_l;
     const float w0 = half == 0 ? w_self : w_other;
@@ -831,7 +862,7 @@ __device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tme
       }
     }
     if (half == 0 && row_ok && p.lse != nullptr)
-      p.lse[static_cast<size_t>(bh) * p.N + q_idx] = (m_ref + __log2f(l_row)) * LN2;
+      p.lse[static_cast<size_t>(bh) * p.N + q_idx] = (m_ref + __log2f(lx_row)) * LN2;
     tc_fence_before();
     g += n;
   }
