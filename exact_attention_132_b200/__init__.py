@@ -18,7 +18,8 @@ import torch
 __all__ = [
     "FAError", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_size", "fa_last_error_string",
     "fa_get_device_status", "fa_debug_wait_timeout_selftest", "fa_version", "fa_fwd_kernel_name",
-    "fa_decode", "fa_decode_workspace_size", "attention_forward", "attention_decode",
+    "fa_decode", "fa_decode_workspace_size", "fa_fwd_gqa", "fa_bwd_gqa", "attention_forward",
+    "attention_decode", "attention_forward_gqa", "attention_backward_gqa",
     "attention_forward_fp8", "attention_backward", "LIB_PATH", "lib",
 ]
 
@@ -53,6 +54,10 @@ def _load() -> ctypes.CDLL:
     L.fa_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     L.fa_debug_wait_timeout_selftest.argtypes = [i, vp]
     L.fa_version.argtypes = []
+    L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    L.fa_fwd_gqa.restype = ctypes.c_int
+    L.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, vp]
+    L.fa_bwd_gqa.restype = ctypes.c_int
     L.fa_decode_workspace_size.argtypes = [i, i, i, i, i, i]
     L.fa_decode_workspace_size.restype = sz
     L.fa_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
@@ -265,3 +270,61 @@ def attention_decode(q, k, v, causal: bool = False, scale: float | None = None):
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     fa_decode(q, k, v, o, lse, ws, scale=scale, causal=causal)
     return o, lse
+
+
+# ------------------------------------------------------------------ grouped heads, full length
+def _gqa_shapes(q, k):
+    B, Hq, N, d = _bhnd(q, "q", torch.bfloat16)
+    Bk, Hkv, Nk, dk = _bhnd(k, "k", torch.bfloat16)
+    if (Bk, Nk, dk) != (B, N, d):
+        raise ValueError("k must be [B, Hkv, N, d] with q's B, N and d")
+    return B, Hq, Hkv, N, d
+
+
+def fa_fwd_gqa(q, k, v, o, lse, scale: float | None = None, causal: bool = False, stream=None):
+    """Forward with Hq query heads on Hkv key/value heads (query head h reads h // g)."""
+    B, Hq, Hkv, N, d = _gqa_shapes(q, k)
+    if _bhnd(v, "v", torch.bfloat16) != (B, Hkv, N, d):
+        raise ValueError("v shape differs from k")
+    if _bhnd(o, "o", torch.bfloat16) != (B, Hq, N, d):
+        raise ValueError("o shape differs from q")
+    if lse is not None and (tuple(lse.shape) != (B, Hq, N) or lse.dtype != torch.float32):
+        raise ValueError("lse must be fp32 [B, Hq, N]")
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.fa_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, sc,
+                          1 if causal else 0, _stream(stream)))
+
+
+def fa_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, workspace, scale: float | None = None,
+               causal: bool = False, stream=None):
+    """Backward with grouped heads; dk, dv sum over the query heads of each group."""
+    B, Hq, Hkv, N, d = _gqa_shapes(q, k)
+    for t, n, h in ((v, "v", Hkv), (o, "o", Hq), (dO, "dO", Hq), (dq, "dq", Hq), (dk, "dk", Hkv),
+                    (dv, "dv", Hkv)):
+        if _bhnd(t, n, torch.bfloat16) != (B, h, N, d):
+            raise ValueError(f"{n} has the wrong shape")
+    if tuple(lse.shape) != (B, Hq, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be fp32 [B, Hq, N]")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.fa_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq),
+                          _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, B, Hq, Hkv, N, d, sc,
+                          1 if causal else 0, _stream(stream)))
+
+
+def attention_forward_gqa(q, k, v, causal: bool = False, scale: float | None = None):
+    """Allocate O and LSE with torch and run fa_fwd_gqa; returns (o, lse)."""
+    B, Hq, N, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    fa_fwd_gqa(q, k, v, o, lse, scale=scale, causal=causal)
+    return o, lse
+
+
+def attention_backward_gqa(q, k, v, o, dO, lse, causal: bool = False, scale: float | None = None):
+    """Allocate dQ/dK/dV and the workspace and run fa_bwd_gqa; returns (dq, dk, dv)."""
+    B, Hq, N, d = q.shape
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(fa_bwd_workspace_size(B, Hq, N, d), 16), dtype=torch.uint8, device=q.device)
+    fa_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, ws, scale=scale, causal=causal)
+    return dq, dk, dv

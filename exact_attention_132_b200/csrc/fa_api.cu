@@ -157,8 +157,8 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, FwdParams p, c
   if (fa_status s = device_info(&di)) return s;
   CUtensorMap mq, mk, mv;
   if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
-  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
-  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
+  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
   auto kern = fa_fwd_kernel<C>;
   if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
   p.n_qt = (p.N + C::BM - 1) / C::BM;
@@ -183,8 +183,8 @@ fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p
   if (fa_status s = device_info(&di)) return s;
   CUtensorMap mq, mk, mv;
   if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
-  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
-  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
+  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
   auto kern = fa_fwd_pp_kernel<C>;
   if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
   {
@@ -220,8 +220,8 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
   if (fa_status s = device_info(&di)) return s;
   CUtensorMap mq, mk, mv;
   if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
-  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
-  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH, C::BN)) return s;
+  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
   auto kern = [] {
     if constexpr (C::SEPARATE_P)
       return fa_fwd_sp_kernel<C>;
@@ -375,14 +375,15 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     CUtensorMap mq, mk, mv, mdo;
     if (fa_status s = make_map(&mq, q, false, D, p.N, p.BH, CK::BMQ)) return s;
     if (fa_status s = make_map(&mdo, dO, false, D, p.N, p.BH, CK::BMQ)) return s;
-    if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH, CK::BN)) return s;
-    if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH, CK::BN)) return s;
+    if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH / p.g, CK::BN)) return s;
+    if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH / p.g, CK::BN)) return s;
     auto kern = fa_bwd_dkdv<CK>;
     if (fa_status s = prepare_kernel<CK>(kern, CK::SMEM_ALLOC)) return s;
     BwdParams pk = p;
     pk.n_qt = (p.N + CK::BMQ - 1) / CK::BMQ;
     pk.n_kt = (p.N + CK::BN - 1) / CK::BN;
-    const long long grid = static_cast<long long>(p.BH) * pk.n_kt * CK::NSPLIT;
+    // one CTA per key/value head, key tile and d part
+    const long long grid = static_cast<long long>(p.BH / p.g) * pk.n_kt * CK::NSPLIT;
     kern<<<static_cast<unsigned>(grid), CK::THREADS, CK::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, pk);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "dK/dV kernel launch");
@@ -392,8 +393,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     CUtensorMap mq, mk, mv, mdo;
     if (fa_status s = make_map(&mq, q, false, D, p.N, p.BH, CQ::BM)) return s;
     if (fa_status s = make_map(&mdo, dO, false, D, p.N, p.BH, CQ::BM)) return s;
-    if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH, CQ::BN)) return s;
-    if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH, CQ::BN)) return s;
+    if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH / p.g, CQ::BN)) return s;
+    if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH / p.g, CQ::BN)) return s;
     auto kern = fa_bwd_dq<CQ>;
     if (fa_status s = prepare_kernel<CQ>(kern, CQ::SMEM_ALLOC)) return s;
     BwdParams pq = p;
@@ -540,19 +541,23 @@ using namespace fa;
 
 extern "C" {
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-                 int d, float scale, int causal, void* stream) {
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                     int Hkv, int N, int d, float scale, int causal, void* stream) {
   bool empty = false;
-  if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
+  if (fa_status s = check_common(B, Hq, N, scale, &empty)) return s;
   if (d != 64 && d != 128 && d != 256)
     return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
   if (empty) return FA_OK;
+  if (Hkv <= 0 || Hq % Hkv != 0)
+    return fail(FA_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d", Hq, Hkv);
   const void* ptrs[] = {q, k, v, o};
   const char* names[] = {"q", "k", "v", "o"};
   if (fa_status s = check_ptrs(ptrs, names, 4)) return s;
   if (lse && !aligned16(lse)) return fail(FA_ERR_INVALID_ARG, "lse is not 16-byte aligned");
   FwdParams p{};
-  p.BH = B * H;
+  p.BH = B * Hq;
+  p.H = Hq;
+  p.g = Hq / Hkv;
   p.N = N;
   p.causal = causal ? 1 : 0;
   p.scale = scale;
@@ -564,6 +569,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     case 128: return FwdD128::launch(q, k, v, p, st);
     default: return launch_fwd<FwdD256>(q, k, v, p, st);
   }
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                 int d, float scale, int causal, void* stream) {
+  return fa_fwd_gqa(q, k, v, o, lse, B, H, H > 0 ? H : 1, N, d, scale, causal, stream);
 }
 
 fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,
@@ -583,6 +593,8 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
   if (lse && !aligned16(lse)) return fail(FA_ERR_INVALID_ARG, "lse is not 16-byte aligned");
   FwdParams p{};
   p.BH = B * H;
+  p.H = H;
+  p.g = 1;
   p.N = N;
   p.causal = causal ? 1 : 0;
   p.scale = scale;
@@ -600,23 +612,27 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return workspace_bytes(B, H, N);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
-                 const float* lse, void* dq, void* dk, void* dv, void* workspace,
-                 size_t workspace_bytes_, int B, int H, int N, int d, float scale, int causal,
-                 void* stream) {
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                     const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                     size_t workspace_bytes_, int B, int Hq, int Hkv, int N, int d, float scale,
+                     int causal, void* stream) {
   bool empty = false;
-  if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
+  if (fa_status s = check_common(B, Hq, N, scale, &empty)) return s;
   if (d != 64 && d != 128 && d != 256)
     return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
   if (empty) return FA_OK;
+  if (Hkv <= 0 || Hq % Hkv != 0)
+    return fail(FA_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d", Hq, Hkv);
   const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv, workspace};
   const char* names[] = {"q", "k", "v", "o", "dO", "lse", "dq", "dk", "dv", "workspace"};
   if (fa_status s = check_ptrs(ptrs, names, 10)) return s;
-  if (workspace_bytes_ < workspace_bytes(B, H, N))
+  if (workspace_bytes_ < workspace_bytes(B, Hq, N))
     return fail(FA_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes_,
-                workspace_bytes(B, H, N));
+                workspace_bytes(B, Hq, N));
   BwdParams p{};
-  p.BH = B * H;
+  p.BH = B * Hq;
+  p.H = Hq;
+  p.g = Hq / Hkv;
   p.N = N;
   p.causal = causal ? 1 : 0;
   p.scale = scale;
@@ -631,6 +647,14 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     case 128: return launch_bwd<DkdvD128, DqD128>(q, k, v, o, dO, p, st);
     default: return launch_bwd<DkdvD256, DqD256>(q, k, v, o, dO, p, st);
   }
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes_, int B, int H, int N, int d, float scale, int causal,
+                 void* stream) {
+  return fa_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes_, B, H,
+                    H > 0 ? H : 1, N, d, scale, causal, stream);
 }
 
 // Same kernels and results as fa_bwd, but the per-row D_i scratch comes from the
@@ -659,6 +683,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if (fa_status s = noalloc_scratch(&scratch)) return s;
   BwdParams p{};
   p.BH = B * H;
+  p.H = H;
+  p.g = 1;
   p.N = N;
   p.causal = causal ? 1 : 0;
   p.scale = scale;

@@ -31,7 +31,9 @@
 namespace fa {
 
 struct BwdParams {
-  int BH, N;
+  int BH, N;             // BH = B * H query heads
+  int H;                 // query heads per batch entry
+  int g;                 // query heads per key/value head (1 = one K/V head per query head)
   int n_qt;              // query tiles of BMQ rows (dK/dV pass) / 128 rows (dQ pass)
   int n_kt;              // key tiles
   int causal;
@@ -203,14 +205,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const float LOG2E = 1.4426950408889634f;
 
-  // block -> (bh, key tile, d part); heaviest causal tiles (small kt) first
+  // block -> (key/value head, key tile, d part); heaviest causal tiles (small kt) first.
+  // With grouped heads the g query heads reading this K/V head all contribute to its
+  // dK, dV: the steps run over (query head of the group, query tile).
   const int split = blockIdx.x % C::NSPLIT;
   const int rest = blockIdx.x / C::NSPLIT;
   const int kt = rest % p.n_kt;
-  const int bh = rest / p.n_kt;
+  const int bh = rest / p.n_kt;                       // key/value head (b * H / g + h / g)
   int i0, i1;
   dkdv_q_range<C>(p, kt, i0, i1);
-  const int nsteps = i1 - i0;
+  const int nqt = i1 - i0;                            // query tiles per query head
+  const int nsteps = nqt * p.g;
+  const int hkv_per_b = p.H / p.g;
+  const int bq0 = (bh / hkv_per_b) * p.H + (bh % hkv_per_b) * p.g;   // first query head
+  // step -> (query head, query tile index)
+  auto q_head = [&](int st) { return bq0 + st / nqt; };
+  auto q_tile = [&](int st) { return i0 + st % nqt; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i) {
@@ -250,16 +260,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     auto fetch = [&](int st) {
 #pragma unroll
       for (int i = 0; i < PL; ++i) {
-        const int q = (i0 + st) * C::BMQ + lane + 32 * i;
+        const int q = q_tile(st) * C::BMQ + lane + 32 * i;
         const bool in = q < p.N;
-        lse_n[i] = in ? p.lse[static_cast<size_t>(bh) * p.N + q] * LOG2E : 0.f;
-        dd_n[i] = in ? p.drow[static_cast<size_t>(bh) * p.N + q] : 0.f;
+        const size_t hq = static_cast<size_t>(q_head(st));
+        lse_n[i] = in ? p.lse[hq * p.N + q] * LOG2E : 0.f;
+        dd_n[i] = in ? p.drow[hq * p.N + q] : 0.f;
       }
     };
     if (nsteps > 0) fetch(0);
     int nq = 0, no = 0;                      // tiles issued per ring
     for (int st = 0; st < nsteps && ok; ++st) {
-      const int qi = i0 + st;
+      const int qi = q_tile(st), hq = q_head(st);
       const int so = st % C::OST, sq = st % C::QST;
       float lse_c[PL], dd_c[PL];
 #pragma unroll
@@ -278,7 +289,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bar(C::B_QFULL + sq), C::QT_BYTES);
         for (int c = 0; c < C::NBOX; ++c)
           tma_load_3d(sbase + C::SMEM_Q + sq * C::QT_BYTES + c * C::BMQ * 128, &tq,
-                      bar(C::B_QFULL + sq), c * 64, qi * C::BMQ, bh);
+                      bar(C::B_QFULL + sq), c * 64, qi * C::BMQ, hq);
       }
       __syncwarp();
       ++nq;
@@ -292,7 +303,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bar(C::B_OFULL + so), C::QT_BYTES);
         for (int c = 0; c < C::NBOX; ++c)
           tma_load_3d(sbase + C::SMEM_DO + so * C::QT_BYTES + c * C::BMQ * 128, &tdo,
-                      bar(C::B_OFULL + so), c * 64, qi * C::BMQ, bh);
+                      bar(C::B_OFULL + so), c * 64, qi * C::BMQ, hq);
       }
       __syncwarp();
       ++no;
@@ -399,7 +410,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const float sl2 = p.scale * LOG2E;
     bool ok = true;
     for (int st = 0; st < nsteps && ok; ++st) {
-      const int qi = i0 + st;
+      const int qi = q_tile(st);
       const int c_first = qi * C::BMQ + half * C::CH;      // first query of this half
       // lse_i and D_i come with their rings' tiles (and are in place once they are)
       if (!(ok = mbar_wait(bar(C::B_QFULL + st % C::QST), (st / C::QST) & 1, wc, kSiteQFull))) break;
@@ -578,6 +589,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   // block -> (bh, q tile); highest causal q tile (most key tiles) first
   const int bh = blockIdx.x / p.n_qt;
+  const int bkv = p.g == 1 ? bh : (bh / p.H) * (p.H / p.g) + (bh % p.H) / p.g;   // K/V head
   const int qt = p.n_qt - 1 - (blockIdx.x - bh * p.n_qt);
   const int nsteps = p.causal ? min(p.n_kt, ((qt + 1) * C::BM - 1) / C::BN + 1) : p.n_kt;
 
@@ -619,7 +631,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bar(C::B_KFULL + sk), C::KT_BYTES);
         for (int c = 0; c < C::NBOX; ++c)
           tma_load_3d(sbase + C::SMEM_K + sk * C::KT_BYTES + c * C::BN * 128, &tk,
-                      bar(C::B_KFULL + sk), c * 64, j * C::BN, bh);
+                      bar(C::B_KFULL + sk), c * 64, j * C::BN, bkv);
       }
       __syncwarp();
       ++nk;
@@ -630,7 +642,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bar(C::B_VFULL + sv), C::KT_BYTES);
         for (int c = 0; c < C::NBOX; ++c)
           tma_load_3d(sbase + C::SMEM_V + sv * C::KT_BYTES + c * C::BN * 128, &tv,
-                      bar(C::B_VFULL + sv), c * 64, j * C::BN, bh);
+                      bar(C::B_VFULL + sv), c * 64, j * C::BN, bkv);
       }
       __syncwarp();
       ++nv;

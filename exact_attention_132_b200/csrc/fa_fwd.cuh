@@ -38,7 +38,9 @@
 namespace fa {
 
 struct FwdParams {
-  int BH;             // B * H
+  int BH;             // B * H (query heads)
+  int H;              // query heads per batch entry
+  int g;              // query heads per key/value head (1 = one K/V head per query head)
   int N;              // sequence length (queries = keys)
   int n_qt;           // ceil(N / 128)
   int n_kt;           // ceil(N / BN)
@@ -55,6 +57,14 @@ struct FwdParams {
   unsigned* status;
   unsigned long long timeout_ns;
 };
+
+// Key/value head of query head `bh` (flattened b * H + h): K/V hold H / g heads per
+// batch entry and query head h reads K/V head h / g.
+__device__ __forceinline__ int fwd_kv_head(const FwdParams& p, int bh) {
+  if (p.g == 1) return bh;
+  const int b = bh / p.H;
+  return b * (p.H / p.g) + (bh - b * p.H) / p.g;
+}
 
 template <int D_, int BN_, int KST_, int VST_, bool FP8_, int EMU_ = 1>
 struct FwdCfg {
@@ -182,9 +192,10 @@ __device__ void fwd_producer(const CUtensorMap* tq, const CUtensorMap* tk, const
       tma_load_3d(sbase + C::SMEM_Q + c * C::BM * 128, tq, bar(C::B_QFULL), c * C::BOX_ELEMS,
                   qt * C::BM, bh);
     ++t;
-    if (!(ok = load_k(0, bh))) break;
-    for (int j = 1; j < n && ok; ++j) ok = load_k(j, bh) && load_v(j - 1, bh);
-    if (ok) ok = load_v(n - 1, bh);
+    const int kvh = fwd_kv_head(p, bh);
+    if (!(ok = load_k(0, kvh))) break;
+    for (int j = 1; j < n && ok; ++j) ok = load_k(j, kvh) && load_v(j - 1, kvh);
+    if (ok) ok = load_v(n - 1, kvh);
   }
   if (!ok) {
     // Aborted: let the tile copies already issued land before the CTA exits.
@@ -330,7 +341,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
       // vmax = largest V tile scale among the visited key tiles; every thread reads
       // the same few values (L1 broadcast), so no cross-warp barrier is needed.
       vmax = 0.f;
-      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[bh * p.n_st + j]);
+      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[fwd_kv_head(p, bh) * p.n_st + j]);
     }
 
     for (int j = 0; j < n; ++j) {
@@ -363,8 +374,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
       float c_j = sl2;
       float fold = 1.f;
       if constexpr (C::FP8) {
-        c_j = sl2 * qsc * p.k_scale[bh * p.n_st + j];
-        fold = 256.f * p.v_scale[bh * p.n_st + j] / vmax;
+        c_j = sl2 * qsc * p.k_scale[fwd_kv_head(p, bh) * p.n_st + j];
+        fold = 256.f * p.v_scale[fwd_kv_head(p, bh) * p.n_st + j] / vmax;
       }
       // row max: four independent three-input chains
       float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;

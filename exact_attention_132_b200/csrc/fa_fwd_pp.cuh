@@ -167,7 +167,7 @@ __device__ void pp_producer(const CUtensorMap* tq, const CUtensorMap* tk, const 
 #pragma unroll
         for (int c = 0; c < C::NBOX; ++c)
           tma_load_3d(sbase + C::SMEM_V + s * C::KV_BYTES + c * C::BN * 128, tv, b_vfull + 8u * s,
-                      c * C::BOX_ELEMS, (j - 1) * C::BN, bh);
+                      c * C::BOX_ELEMS, (j - 1) * C::BN, fwd_kv_head(p, bh));
         ++gv;
       }
       if (j < ns) {
@@ -180,7 +180,7 @@ __device__ void pp_producer(const CUtensorMap* tq, const CUtensorMap* tk, const 
 #pragma unroll
         for (int c = 0; c < C::NBOX; ++c)
           tma_load_3d(sbase + C::SMEM_K + s * C::KV_BYTES + c * C::BN * 128, tk, b_kfull + 8u * s,
-                      c * C::BOX_ELEMS, j * C::BN, bh);
+                      c * C::BOX_ELEMS, j * C::BN, fwd_kv_head(p, bh));
         ++gk;
       }
     }
@@ -326,21 +326,21 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
     // overlaps the wait for the scores
     float ksc_n = 1.f, vsc_n = 1.f;
     if constexpr (C::FP8) {
-      const float* vs = p.v_scale + bh * p.n_st;
+      const float* vs = p.v_scale + fwd_kv_head(p, bh) * p.n_st;
       qsc = p.q_scale[bh * p.n_st + qt];
       vmax = 0.f;
       for (int j = threadIdx.x & 31; j < n; j += 32) vmax = fmaxf(vmax, vs[j]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
-      ksc_n = p.k_scale[bh * p.n_st];
+      ksc_n = p.k_scale[fwd_kv_head(p, bh) * p.n_st];
       vsc_n = vs[0];
     }
     for (int j = 0; j < n; ++j) {
       const float ksc = ksc_n, vsc = vsc_n;
       if constexpr (C::FP8) {
         if (j + 1 < n) {
-          ksc_n = p.k_scale[bh * p.n_st + j + 1];
-          vsc_n = p.v_scale[bh * p.n_st + j + 1];
+          ksc_n = p.k_scale[fwd_kv_head(p, bh) * p.n_st + j + 1];
+          vsc_n = p.v_scale[fwd_kv_head(p, bh) * p.n_st + j + 1];
         }
       }
       if (!(ok = mbar_wait(bar(C::B_SFULL + t), gs & 1, wc, kSiteSFull))) break;

@@ -322,7 +322,7 @@ __device__ void sp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, flo
     if constexpr (C::FP8) {
       qsc = p.q_scale[bh * p.n_st + qt];
       vmax = 0.f;
-      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[bh * p.n_st + j]);
+      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[fwd_kv_head(p, bh) * p.n_st + j]);
     }
     for (int j = 0; j < n; ++j) {
       const uint32_t gj = g + j;
@@ -351,8 +351,8 @@ __device__ void sp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, flo
       }
       float c_j = sl2, fold = 1.f;
       if constexpr (C::FP8) {
-        c_j = sl2 * qsc * p.k_scale[bh * p.n_st + j];
-        fold = 256.f * p.v_scale[bh * p.n_st + j] / vmax;
+        c_j = sl2 * qsc * p.k_scale[fwd_kv_head(p, bh) * p.n_st + j];
+        fold = 256.f * p.v_scale[fwd_kv_head(p, bh) * p.n_st + j] / vmax;
       }
       float mx[8];
 #pragma unroll

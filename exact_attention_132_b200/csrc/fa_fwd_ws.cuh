@@ -154,7 +154,7 @@ __device__ void ws_producer(const CUtensorMap* tq, const CUtensorMap* tk, const 
 #pragma unroll
           for (int c = 0; c < C::NBOX; ++c)
             tma_load_3d(sbase + C::SMEM_K + s * C::KV_BYTES + c * C::BN * 128, tk, b_kfull + 8u * s,
-                        c * C::BOX_ELEMS, j * C::BN, bh);
+                        c * C::BOX_ELEMS, j * C::BN, fwd_kv_head(p, bh));
         }
         __syncwarp();
         ++gk;
@@ -171,7 +171,7 @@ __device__ void ws_producer(const CUtensorMap* tq, const CUtensorMap* tk, const 
 #pragma unroll
           for (int c = 0; c < C::NBOX; ++c)
             tma_load_3d(sbase + C::SMEM_V + s * C::KV_BYTES + c * C::BN * 128, tv, b_vfull + 8u * s,
-                        c * C::BOX_ELEMS, (j - 1) * C::BN, bh);
+                        c * C::BOX_ELEMS, (j - 1) * C::BN, fwd_kv_head(p, bh));
         }
         __syncwarp();
         ++gv;
@@ -391,7 +391,7 @@ __device__ void ws_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, flo
     if constexpr (C::FP8) {
       qsc = p.q_scale[bh * p.n_st + qt];
       vmax = 0.f;
-      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[bh * p.n_st + j]);
+      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[fwd_kv_head(p, bh) * p.n_st + j]);
     }
     for (int j = 0; j < n; ++j) {
       const uint32_t gj = g + j;
@@ -416,8 +416,8 @@ __device__ void ws_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, flo
       }
       float c_j = sl2, fold = 1.f;
       if constexpr (C::FP8) {
-        c_j = sl2 * qsc * p.k_scale[bh * p.n_st + j];
-        fold = 256.f * p.v_scale[bh * p.n_st + j] / vmax;
+        c_j = sl2 * qsc * p.k_scale[fwd_kv_head(p, bh) * p.n_st + j];
+        fold = 256.f * p.v_scale[fwd_kv_head(p, bh) * p.n_st + j] / vmax;
       }
       float mx[4];
 #pragma unroll
@@ -694,7 +694,7 @@ __device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tme
     if constexpr (C::FP8) {
       qsc = p.q_scale[bh * p.n_st + qt];
       vmax = 0.f;
-      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[bh * p.n_st + j]);
+      for (int j = 0; j < n; ++j) vmax = fmaxf(vmax, p.v_scale[fwd_kv_head(p, bh) * p.n_st + j]);
     }
     for (int j = 0; j < n; ++j) {
       const uint32_t gj = g + j;
@@ -722,8 +722,8 @@ __device__ void ws_softmax_indep(const FwdParams& p, uint32_t bars, uint32_t tme
       }
       float c_j = sl2, fold = 1.f;
       if constexpr (C::FP8) {
-        c_j = sl2 * qsc * p.k_scale[bh * p.n_st + j];
-        fold = 256.f * p.v_scale[bh * p.n_st + j] / vmax;
+        c_j = sl2 * qsc * p.k_scale[fwd_kv_head(p, bh) * p.n_st + j];
+        fold = 256.f * p.v_scale[fwd_kv_head(p, bh) * p.n_st + j] / vmax;
       }
       float mx[4];
 #pragma unroll

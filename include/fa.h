@@ -149,6 +149,24 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * Grouped query heads (GQA / MQA, "FlashAttention — フラッシュアテンション"
+ * (systems-analysis.info), section FlashAttention-2（2023年）) for the full-length
+ * forward and backward: Hq query heads share Hkv key/value heads, query head h reads
+ * key/value head h / (Hq / Hkv).
+ *   q, o, dO, dq     bf16 [B, Hq, N, d];  k, v, dk, dv  bf16 [B, Hkv, N, d];
+ *   lse              fp32 [B, Hq, N];     workspace     >= fa_bwd_workspace_size(B, Hq, N, d)
+ * dk, dv sum the contributions of every query head of the group.  Hq % Hkv must be
+ * 0 (FA_ERR_INVALID_ARG otherwise).  Everything else as fa_fwd / fa_bwd, which are
+ * these calls with Hkv = Hq.
+ */
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int N, int d, float scale, int causal, void* stream);
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                     const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                     size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
+                     int causal, void* stream);
+
+/*
  * Decoding: few query rows against a long key/value sequence, with grouped query
  * heads (GQA / MQA).  Same exact attention as fa_fwd.  Decoding reads Q of length 1
  * against the whole KV cache, so reading K and V bounds it ("FlashAttentionとは？…"

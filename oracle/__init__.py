@@ -1,6 +1,7 @@
 """fp64 CPU oracle (test infrastructure only; never imported by the product path)."""
 from .attention_ref import (  # noqa: F401
     attention_bwd,
+    attention_bwd_gqa,
     attention_bwd_rows_dq,
     attention_decode,
     attention_fwd,

@@ -284,3 +284,29 @@ def attention_decode(q, k, v, scale: float, causal: bool):
             O[b, h] = (e / l) @ v[b, h // g]
             L[b, h] = (m + np.log(l))[:, 0]
     return O, L
+
+
+def attention_bwd_gqa(q, k, v, do, scale: float, causal: bool):
+    """dQ, dK, dV in fp64 with grouped heads: q, do [B, Hq, N, d]; k, v [B, Hkv, N, d].
+
+    Query head h attends through key/value head h // g (g = Hq / Hkv; "FlashAttention —
+    フラッシュアテンション" (systems-analysis.info), section FlashAttention-2（2023年）).
+    A shared K/V head is used by g attention computations, so by the chain rule its
+    gradient is the sum of the g per-use gradients; each use is the one-head backward
+    above (materialised P, no saved LSE).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Hq = q.shape[:2]
+    Hkv = k.shape[1]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    g = Hq // Hkv
+    dq = np.empty_like(q)
+    dk, dv = np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // g
+            dq[b, h], dkh, dvh = _head_bwd(q[b, h], k[b, hk], v[b, hk], do[b, h], scale, causal)
+            dk[b, hk] += dkh
+            dv[b, hk] += dvh
+    return dq, dk, dv

@@ -345,3 +345,43 @@ def check_dec_last_query_sees_all(dec) -> bool:
 
 DEC_CHECKS = [check_dec_brute, check_dec_q_zero, check_dec_constant_v, check_dec_torch_sdpa,
               check_dec_square_is_forward, check_dec_last_query_sees_all]
+
+
+# --------------------------------------------------------------------------- grouped-head backward
+# bwd_gqa signature: bwd(q [B,Hq,N,d], k [B,Hkv,N,d], v, do, scale, causal) -> (dQ, dK, dV)
+def check_gqa_bwd_torch_autograd(bwd) -> bool:
+    """fp64 autograd through torch SDPA with the key/value heads repeated per group:
+    autograd itself sums the gradients of the repeated (shared) heads."""
+    r = _rng(47)
+    B, Hq, Hkv, N, d = 2, 6, 2, 11, 5
+    q = r.standard_normal((B, Hq, N, d))
+    k, v = (r.standard_normal((B, Hkv, N, d)) for _ in range(2))
+    do = r.standard_normal((B, Hq, N, d))
+    ok = True
+    for causal in (False, True):
+        tq, tk, tv = (torch.from_numpy(x).requires_grad_(True) for x in (q, k, v))
+        o = torch.nn.functional.scaled_dot_product_attention(
+            tq, tk.repeat_interleave(Hq // Hkv, dim=1), tv.repeat_interleave(Hq // Hkv, dim=1),
+            is_causal=causal, scale=0.37)
+        o.backward(torch.from_numpy(do))
+        dq, dk, dv = bwd(q, k, v, do, 0.37, causal)
+        ok &= _close(dq, tq.grad.numpy(), 1e-11) and _close(dk, tk.grad.numpy(), 1e-11) \
+            and _close(dv, tv.grad.numpy(), 1e-11)
+    return ok
+
+
+def check_gqa_bwd_one_group_is_mha(bwd) -> bool:
+    """g = 1 is the ordinary backward: scalar brute force per head."""
+    r = _rng(53)
+    q, k, v, do = (r.standard_normal((1, 2, 6, 3)) for _ in range(4))
+    ok = True
+    for causal in (False, True):
+        dq, dk, dv = bwd(q, k, v, do, 0.8, causal)
+        for h in range(2):
+            bq, bk, bv = brute_bwd(q[0, h].tolist(), k[0, h].tolist(), v[0, h].tolist(),
+                                   do[0, h].tolist(), 0.8, causal)
+            ok &= _close(dq[0, h], bq, 1e-12) and _close(dk[0, h], bk, 1e-12) and _close(dv[0, h], bv, 1e-12)
+    return ok
+
+
+GQA_BWD_CHECKS = [check_gqa_bwd_torch_autograd, check_gqa_bwd_one_group_is_mha]

@@ -169,3 +169,40 @@ def test_decode_mutant_is_caught(name):
         if not ok:
             failures.append(chk.__name__)
     assert failures, f"mutant {name} passed every decoding check"
+
+
+# ----------------------------------------------------------------------------- grouped-head backward
+def _gqa_bwd_generic(q, k, v, do, scale, causal, *, last_only=False, head_mod=False):
+    q, k, v, do = (np.asarray(x, dtype=np.float64) for x in (q, k, v, do))
+    B, Hq = q.shape[:2]
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    dq = np.empty_like(q)
+    dk, dv = np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h % Hkv if head_mod else h // g
+            a, bk, bv = oracle.attention_bwd(q[b:b + 1, h:h + 1], k[b:b + 1, hk:hk + 1],
+                                             v[b:b + 1, hk:hk + 1], do[b:b + 1, h:h + 1], scale, causal)
+            dq[b, h] = a[0, 0]
+            if last_only:
+                dk[b, hk], dv[b, hk] = bk[0, 0], bv[0, 0]
+            else:
+                dk[b, hk] += bk[0, 0]
+                dv[b, hk] += bv[0, 0]
+    return dq, dk, dv
+
+
+MUTANTS_GQA_BWD = {"shared_grad_not_summed": dict(last_only=True), "kv_head_modulo": dict(head_mod=True)}
+
+
+def test_unmutated_gqa_backward_passes():
+    for chk in oc.GQA_BWD_CHECKS:
+        assert chk(_gqa_bwd_generic), chk.__name__
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS_GQA_BWD))
+def test_gqa_backward_mutant_is_caught(name):
+    kw = MUTANTS_GQA_BWD[name]
+    f = lambda q, k, v, do, s, c: _gqa_bwd_generic(q, k, v, do, s, c, **kw)
+    assert not all(chk(f) for chk in oc.GQA_BWD_CHECKS), f"mutant {name} passed every check"

@@ -88,3 +88,8 @@ def test_row_blocking_is_exact(monkeypatch):
 @pytest.mark.parametrize("check", oc.DEC_CHECKS, ids=lambda f: f.__name__)
 def test_oracle_decode_pins(check):
     assert check(oracle.attention_decode)
+
+
+@pytest.mark.parametrize("check", oc.GQA_BWD_CHECKS, ids=lambda f: f.__name__)
+def test_oracle_gqa_backward_pins(check):
+    assert check(oracle.attention_bwd_gqa)
