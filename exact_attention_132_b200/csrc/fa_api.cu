@@ -156,9 +156,9 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, FwdParams p, c
   DeviceInfo* di = nullptr;
   if (fa_status s = device_info(&di)) return s;
   CUtensorMap mq, mk, mv;
-  if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
-  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
-  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
+  if (fa_status s = make_map(&mq, q, C::FP8, p.ld, p.N, p.BH, C::BM)) return s;
+  if (fa_status s = make_map(&mk, k, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
   auto kern = fa_fwd_kernel<C>;
   if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
   p.n_qt = (p.N + C::BM - 1) / C::BM;
@@ -182,9 +182,9 @@ fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p
   DeviceInfo* di = nullptr;
   if (fa_status s = device_info(&di)) return s;
   CUtensorMap mq, mk, mv;
-  if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
-  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
-  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
+  if (fa_status s = make_map(&mq, q, C::FP8, p.ld, p.N, p.BH, C::BM)) return s;
+  if (fa_status s = make_map(&mk, k, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
   auto kern = fa_fwd_pp_kernel<C>;
   if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
   {
@@ -219,9 +219,9 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
   DeviceInfo* di = nullptr;
   if (fa_status s = device_info(&di)) return s;
   CUtensorMap mq, mk, mv;
-  if (fa_status s = make_map(&mq, q, C::FP8, C::D, p.N, p.BH, C::BM)) return s;
-  if (fa_status s = make_map(&mk, k, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
-  if (fa_status s = make_map(&mv, v, C::FP8, C::D, p.N, p.BH / p.g, C::BN)) return s;
+  if (fa_status s = make_map(&mq, q, C::FP8, p.ld, p.N, p.BH, C::BM)) return s;
+  if (fa_status s = make_map(&mk, k, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
   auto kern = [] {
     if constexpr (C::SEPARATE_P)
       return fa_fwd_sp_kernel<C>;
@@ -357,26 +357,34 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   constexpr int D = CK::D;
   p.status = di->status;
   p.timeout_ns = kWaitTimeoutNs;
-  // 1. D_i = dO_i . O_i
+  // 1. D_i = dO_i . O_i over the stored head dim
   {
     const long long rows = static_cast<long long>(p.BH) * p.N;
-    constexpr int rpb = 256 / (D / 8);
-    long long blocks = (rows + rpb - 1) / rpb;
-    const long long cap = static_cast<long long>(di->sms) * 8;
-    if (blocks > cap) blocks = cap;
-    fa_bwd_rowdot<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO),
-        const_cast<float*>(p.drow), rows);
+    auto rowdot = [&](auto kern, int rpb) {
+      long long blocks = (rows + rpb - 1) / rpb;
+      const long long cap = static_cast<long long>(di->sms) * 8;
+      if (blocks > cap) blocks = cap;
+      kern<<<static_cast<int>(blocks), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO),
+          const_cast<float*>(p.drow), rows);
+    };
+    static_assert(D == 64 || D == 128 || D == 256, "kernel head dims");
+    if (p.ld == D)
+      rowdot(fa_bwd_rowdot<D>, 256 / (D / 8));
+    else if (p.ld == 96)
+      rowdot(fa_bwd_rowdot<96>, 64);
+    else
+      rowdot(fa_bwd_rowdot<192>, 32);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "row-dot kernel launch");
   }
   // 2. dK, dV
   {
     CUtensorMap mq, mk, mv, mdo;
-    if (fa_status s = make_map(&mq, q, false, D, p.N, p.BH, CK::BMQ)) return s;
-    if (fa_status s = make_map(&mdo, dO, false, D, p.N, p.BH, CK::BMQ)) return s;
-    if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH / p.g, CK::BN)) return s;
-    if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH / p.g, CK::BN)) return s;
+    if (fa_status s = make_map(&mq, q, false, p.ld, p.N, p.BH, CK::BMQ)) return s;
+    if (fa_status s = make_map(&mdo, dO, false, p.ld, p.N, p.BH, CK::BMQ)) return s;
+    if (fa_status s = make_map(&mk, k, false, p.ld, p.N, p.BH / p.g, CK::BN)) return s;
+    if (fa_status s = make_map(&mv, v, false, p.ld, p.N, p.BH / p.g, CK::BN)) return s;
     auto kern = fa_bwd_dkdv<CK>;
     if (fa_status s = prepare_kernel<CK>(kern, CK::SMEM_ALLOC)) return s;
     BwdParams pk = p;
@@ -391,10 +399,10 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   // 3. dQ
   {
     CUtensorMap mq, mk, mv, mdo;
-    if (fa_status s = make_map(&mq, q, false, D, p.N, p.BH, CQ::BM)) return s;
-    if (fa_status s = make_map(&mdo, dO, false, D, p.N, p.BH, CQ::BM)) return s;
-    if (fa_status s = make_map(&mk, k, false, D, p.N, p.BH / p.g, CQ::BN)) return s;
-    if (fa_status s = make_map(&mv, v, false, D, p.N, p.BH / p.g, CQ::BN)) return s;
+    if (fa_status s = make_map(&mq, q, false, p.ld, p.N, p.BH, CQ::BM)) return s;
+    if (fa_status s = make_map(&mdo, dO, false, p.ld, p.N, p.BH, CQ::BM)) return s;
+    if (fa_status s = make_map(&mk, k, false, p.ld, p.N, p.BH / p.g, CQ::BN)) return s;
+    if (fa_status s = make_map(&mv, v, false, p.ld, p.N, p.BH / p.g, CQ::BN)) return s;
     auto kern = fa_bwd_dq<CQ>;
     if (fa_status s = prepare_kernel<CQ>(kern, CQ::SMEM_ALLOC)) return s;
     BwdParams pq = p;
@@ -474,8 +482,8 @@ fa_status dec_check(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, 
     return fail(FA_ERR_INVALID_ARG, "negative size B=%d Hq=%d Hkv=%d Nq=%d Nk=%d", B, Hq, Hkv, Nq, Nk);
   if (!std::isfinite(scale) || !(scale > 0.f))
     return fail(FA_ERR_INVALID_ARG, "scale must be finite and > 0 (got %g)", static_cast<double>(scale));
-  if (d != 64 && d != 128 && d != 256)
-    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
+  if (d != 64 && d != 96 && d != 128 && d != 192 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 96, 128, 192, 256)", d);
   *empty = (B == 0 || Hq == 0 || Nq == 0);
   if (*empty) return FA_OK;
   if (Hkv == 0 || Hq % Hkv != 0)
@@ -496,6 +504,7 @@ fa_status dec_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, DecPlan* pl) {
   pl->BHkv = B * Hkv;
   pl->R = (Hq / Hkv) * Nq;
   pl->bn = d <= 128 ? 128 : 64;
+  const int dk = d <= 64 ? 64 : (d <= 128 ? 128 : 256);   // kernel head dim
   pl->n_kt = (Nk + pl->bn - 1) / pl->bn;
   const long long target = 2ll * di->sms;
   long long ns = (target + pl->BHkv - 1) / pl->BHkv;
@@ -504,7 +513,7 @@ fa_status dec_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, DecPlan* pl) {
   pl->split_tiles = static_cast<int>((pl->n_kt + ns - 1) / ns);
   pl->n_split = (pl->n_kt + pl->split_tiles - 1) / pl->split_tiles;
   const size_t rows = static_cast<size_t>(pl->BHkv) * pl->n_split * pl->R;
-  pl->part_o_bytes = (rows * d * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  pl->part_o_bytes = (rows * dk * sizeof(float) + 255) & ~static_cast<size_t>(255);
   pl->part_lse_bytes = (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
   pl->total = pl->part_o_bytes + pl->part_lse_bytes;
   return FA_OK;
@@ -516,9 +525,9 @@ fa_status launch_decode(const void* q, const void* k, const void* v, void* o, fl
   DeviceInfo* di = nullptr;
   if (fa_status s = device_info(&di)) return s;
   CUtensorMap mq, mk, mv;
-  if (fa_status s = make_map(&mq, q, false, C::D, p.R, p.BHkv, C::BM)) return s;
-  if (fa_status s = make_map(&mk, k, false, C::D, p.Nk, p.BHkv, C::BN)) return s;
-  if (fa_status s = make_map(&mv, v, false, C::D, p.Nk, p.BHkv, C::BN)) return s;
+  if (fa_status s = make_map(&mq, q, false, p.ld, p.R, p.BHkv, C::BM)) return s;
+  if (fa_status s = make_map(&mk, k, false, p.ld, p.Nk, p.BHkv, C::BN)) return s;
+  if (fa_status s = make_map(&mv, v, false, p.ld, p.Nk, p.BHkv, C::BN)) return s;
   auto kern = fa_decode_split_kernel<C>;
   if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
   p.status = di->status;
@@ -545,8 +554,8 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
                      int Hkv, int N, int d, float scale, int causal, void* stream) {
   bool empty = false;
   if (fa_status s = check_common(B, Hq, N, scale, &empty)) return s;
-  if (d != 64 && d != 128 && d != 256)
-    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
+  if (d != 64 && d != 96 && d != 128 && d != 192 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 96, 128, 192, 256)", d);
   if (empty) return FA_OK;
   if (Hkv <= 0 || Hq % Hkv != 0)
     return fail(FA_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d", Hq, Hkv);
@@ -558,14 +567,19 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
   p.BH = B * Hq;
   p.H = Hq;
   p.g = Hq / Hkv;
+  p.ld = d;
   p.N = N;
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.o = o;
   p.lse = lse;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // d = 96 and 192 run on the 128 and 256 kernels: the tensor maps know the true row
+  // length, so the extra columns load as zeros (adding nothing to Q K^T or P V) and the
+  // epilogue stores only the first d
   switch (d) {
     case 64: return FwdD64::launch(q, k, v, p, st);
+    case 96:
     case 128: return FwdD128::launch(q, k, v, p, st);
     default: return launch_fwd<FwdD256>(q, k, v, p, st);
   }
@@ -595,6 +609,7 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
   p.BH = B * H;
   p.H = H;
   p.g = 1;
+  p.ld = d;
   p.N = N;
   p.causal = causal ? 1 : 0;
   p.scale = scale;
@@ -618,8 +633,8 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
                      int causal, void* stream) {
   bool empty = false;
   if (fa_status s = check_common(B, Hq, N, scale, &empty)) return s;
-  if (d != 64 && d != 128 && d != 256)
-    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
+  if (d != 64 && d != 96 && d != 128 && d != 192 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 96, 128, 192, 256)", d);
   if (empty) return FA_OK;
   if (Hkv <= 0 || Hq % Hkv != 0)
     return fail(FA_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d", Hq, Hkv);
@@ -633,6 +648,7 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
   p.BH = B * Hq;
   p.H = Hq;
   p.g = Hq / Hkv;
+  p.ld = d;
   p.N = N;
   p.causal = causal ? 1 : 0;
   p.scale = scale;
@@ -644,6 +660,7 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d) {
     case 64: return launch_bwd<DkdvD64, DqD64>(q, k, v, o, dO, p, st);
+    case 96:
     case 128: return launch_bwd<DkdvD128, DqD128>(q, k, v, o, dO, p, st);
     default: return launch_bwd<DkdvD256, DqD256>(q, k, v, o, dO, p, st);
   }
@@ -668,8 +685,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          float scale, int causal, void* stream) {
   bool empty = false;
   if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
-  if (d != 64 && d != 128 && d != 256)
-    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 128, 256)", d);
+  if (d != 64 && d != 96 && d != 128 && d != 192 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 96, 128, 192, 256)", d);
   if (empty) return FA_OK;
   const long long rows = static_cast<long long>(B) * H * N;
   if (rows > FA_BWD_NOALLOC_MAX_ROWS)
@@ -685,6 +702,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   p.BH = B * H;
   p.H = H;
   p.g = 1;
+  p.ld = d;
   p.N = N;
   p.causal = causal ? 1 : 0;
   p.scale = scale;
@@ -696,6 +714,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d) {
     case 64: return launch_bwd<DkdvD64, DqD64>(q, k, v, o, dO, p, st);
+    case 96:
     case 128: return launch_bwd<DkdvD128, DqD128>(q, k, v, o, dO, p, st);
     default: return launch_bwd<DkdvD256, DqD256>(q, k, v, o, dO, p, st);
   }
@@ -756,6 +775,7 @@ fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float*
   p.R = pl.R;
   p.Nq = Nq;
   p.Nk = Nk;
+  p.ld = d;
   p.causal = causal ? 1 : 0;
   p.n_kt = pl.n_kt;
   p.split_tiles = pl.split_tiles;
@@ -767,6 +787,7 @@ fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d) {
     case 64: return launch_decode<DecD64>(q, k, v, o, lse, p, st);
+    case 96:
     case 128: return launch_decode<DecD128>(q, k, v, o, lse, p, st);
     default: return launch_decode<DecD256>(q, k, v, o, lse, p, st);
   }
@@ -779,7 +800,9 @@ const char* fa_fwd_kernel_name(int head_dim, int fp8) {
   if (fp8) return head_dim == 128 ? FwdF8D128::name() : nullptr;
   switch (head_dim) {
     case 64: return FwdD64::name();
+    case 96:
     case 128: return FwdD128::name();
+    case 192:
     case 256: {
       static const std::string n = "fa_fwd_kernel<FwdCfg<256,KST" + std::to_string(FwdD256::KST) +
                                    ",VST" + std::to_string(FwdD256::VST) + ",bf16>>";

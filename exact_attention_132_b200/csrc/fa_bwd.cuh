@@ -34,6 +34,8 @@ struct BwdParams {
   int BH, N;             // BH = B * H query heads
   int H;                 // query heads per batch entry
   int g;                 // query heads per key/value head (1 = one K/V head per query head)
+  int ld;                // head dim as stored (row length of every bf16 tensor); the kernel's
+                         // D may be larger: columns past ld load as zeros, are not stored
   int n_qt;              // query tiles of BMQ rows (dK/dV pass) / 128 rows (dQ pass)
   int n_kt;              // key tiles
   int causal;
@@ -48,28 +50,35 @@ struct BwdParams {
 };
 
 // --------------------------------------------------------------------------- 1. D_i
-// D_i = sum_c dO_ic * O_ic, fp32 accumulation of the bf16 products.  Each group of
-// D/8 threads reads one row with 16-byte loads.
+// D_i = sum_c dO_ic * O_ic, fp32 accumulation of the bf16 products.  A row of D
+// elements is D/8 16-byte pieces; TPR threads (a power of two) share a row, PER pieces
+// each: D = 64 -> 8 x 1, 128 -> 16 x 1, 256 -> 32 x 1, 96 -> 4 x 3, 192 -> 8 x 3.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_rowdot(const __nv_bfloat16* __restrict__ o,
                                                      const __nv_bfloat16* __restrict__ dout,
                                                      float* __restrict__ drow, long long rows) {
-  constexpr int TPR = D / 8;                 // threads per row
-  constexpr int RPB = 256 / TPR;             // rows per block pass
+  constexpr int PIECES = D / 8;
+  constexpr int PER = (PIECES % 3 == 0) ? 3 : 1;   // pieces per thread
+  constexpr int TPR = PIECES / PER;                  // threads per row
+  static_assert((TPR & (TPR - 1)) == 0 && TPR <= 32, "power-of-two threads per row");
+  constexpr int RPB = 256 / TPR;                     // rows per block pass
   const int sub = threadIdx.x % TPR;
   for (long long r = static_cast<long long>(blockIdx.x) * RPB + threadIdx.x / TPR; r < rows;
        r += static_cast<long long>(gridDim.x) * RPB) {
-    const uint4 a = reinterpret_cast<const uint4*>(o + r * D)[sub];
-    const uint4 b = reinterpret_cast<const uint4*>(dout + r * D)[sub];
-    const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&b);
     float acc = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 fa2 = __bfloat1622float2(ha[i]);
-      const float2 fb2 = __bfloat1622float2(hb[i]);
-      acc = fmaf(fa2.x, fb2.x, acc);
-      acc = fmaf(fa2.y, fb2.y, acc);
+    for (int u = 0; u < PER; ++u) {
+      const uint4 a = reinterpret_cast<const uint4*>(o + r * D)[sub * PER + u];
+      const uint4 b = reinterpret_cast<const uint4*>(dout + r * D)[sub * PER + u];
+      const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 fa2 = __bfloat1622float2(ha[i]);
+        const float2 fb2 = __bfloat1622float2(hb[i]);
+        acc = fmaf(fa2.x, fb2.x, acc);
+        acc = fmaf(fa2.y, fb2.y, acc);
+      }
     }
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -491,7 +500,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_fence_after();
       const bool row_ok = kv < p.N;
       const size_t base =
-          (static_cast<size_t>(bh) * p.N + kv) * C::D + split * C::DH + half * (C::DH / 2);
+          (static_cast<size_t>(bh) * p.N + kv) * p.ld + split * C::DH + half * (C::DH / 2);
+      const int cbase = split * C::DH + half * (C::DH / 2);   // first column written here
       __nv_bfloat16* dvp = reinterpret_cast<__nv_bfloat16*>(p.dv) + base;
       __nv_bfloat16* dkp = reinterpret_cast<__nv_bfloat16*>(p.dk) + base;
 #pragma unroll 1
@@ -508,7 +518,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
-          if (row_ok) {
+          if (row_ok && cbase + c < p.ld) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
             for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
@@ -798,7 +808,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (ok && mbar_wait(bar(C::B_ACC), 0, wc, kSiteDqDone)) {
       tc_fence_after();
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.dq) +
-                           (static_cast<size_t>(bh) * p.N + q) * C::D + half * (C::D / 2);
+                           (static_cast<size_t>(bh) * p.N + q) * p.ld + half * (C::D / 2);
 #pragma unroll 1
       for (int c = 0; c < C::D / 2; c += 32) {
         uint32_t r[32];
@@ -808,7 +818,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
-        if (row_ok) {
+        if (row_ok && half * (C::D / 2) + c < p.ld) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
           for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);

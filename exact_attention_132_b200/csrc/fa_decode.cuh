@@ -37,6 +37,7 @@ struct DecParams {
   int BHkv;            // B * Hkv
   int R;               // query rows per key/value head: (Hq / Hkv) * Nq, <= 128
   int Nq, Nk;
+  int ld;              // head dim as stored (row length of q, k, v, o); D may be larger
   int causal;
   int n_kt;            // ceil(Nk / BN)
   int split_tiles;     // key tiles per split
@@ -418,9 +419,10 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecParams 
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = fmaf(wgt, src[lane + 32 * i], acc[i]);
   }
-  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o) + (static_cast<size_t>(bh) * p.R + row) * D;
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o) + (static_cast<size_t>(bh) * p.R + row) * p.ld;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) dst[lane + 32 * i] = __float2bfloat16_rn(acc[i]);
+  for (int i = 0; i < PER; ++i)
+    if (lane + 32 * i < p.ld) dst[lane + 32 * i] = __float2bfloat16_rn(acc[i]);
   if (lse != nullptr && lane == 0) lse[static_cast<size_t>(bh) * p.R + row] = lse_row;
 }
 

@@ -41,6 +41,8 @@ struct FwdParams {
   int BH;             // B * H (query heads)
   int H;              // query heads per batch entry
   int g;              // query heads per key/value head (1 = one K/V head per query head)
+  int ld;             // head dim as stored (row length of q, k, v, o); the kernel's D may
+                      // be larger: columns past ld load as zeros and are not stored
   int N;              // sequence length (queries = keys)
   int n_qt;           // ceil(N / 128)
   int n_kt;           // ceil(N / BN)
@@ -473,7 +475,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
     tc_fence_after();
     const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / l;
     const bool row_ok = q_idx < p.N;
-    __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * C::D;
+    __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * p.ld;
 #pragma unroll 1
     for (int c = 0; c < C::D; c += 32) {
       uint32_t r[32];
@@ -483,7 +485,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-      if (row_ok) {
+      if (row_ok && c < p.ld) {
         uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
         for (int i = 0; i < 4; ++i)

@@ -509,7 +509,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
     tc_fence_after();
     const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / l;
     const bool row_ok = q_idx < p.N;
-    __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * C::D;
+    __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * p.ld;
 #pragma unroll 1
     for (int c = 0; c < C::D; c += 32) {
       uint32_t r[32];
@@ -519,7 +519,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-      if (row_ok) {
+      if (row_ok && c < p.ld) {
         uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
         for (int i = 0; i < 4; ++i)

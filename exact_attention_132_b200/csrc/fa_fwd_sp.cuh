@@ -443,7 +443,7 @@ __device__ void sp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, flo
     const float w0 = (half == 0 ? e_me : e_ot) * inv_l;
     const float w1 = (half == 0 ? e_ot : e_me) * inv_l;
     const bool row_ok = q_idx < p.N;
-    __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * C::D + half * C::DH;
+    __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * p.ld + half * C::DH;
 #pragma unroll 1
     for (int c = 0; c < C::DH; c += 32) {
       uint32_t a0[32], a1[32];
@@ -458,7 +458,7 @@ __device__ void sp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, flo
         const float y0 = fmaf(__uint_as_float(a1[2 * i + 1]), w1, __uint_as_float(a0[2 * i + 1]) * w0);
         pk[i] = pack_bf16x2(x0, y0);
       }
-      if (row_ok) {
+      if (row_ok && half * C::DH + c < p.ld) {
         uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
         for (int i = 0; i < 4; ++i)

@@ -45,7 +45,10 @@ def test_forward_kernel_names():
         name = fa.fa_fwd_kernel_name(d, fp8)
         assert name and name.startswith("fa_fwd_") and f"<{d}," in name
         assert ("e4m3" in name) == fp8
-    assert fa.fa_fwd_kernel_name(96) is None
+    assert fa.fa_fwd_kernel_name(80) is None
+    # stored head dims 96 and 192 run on the 128 and 256 kernels
+    assert fa.fa_fwd_kernel_name(96) == fa.fa_fwd_kernel_name(128)
+    assert fa.fa_fwd_kernel_name(192) == fa.fa_fwd_kernel_name(256)
     assert fa.fa_fwd_kernel_name(64, True) is None
 
 
@@ -61,7 +64,7 @@ def test_argument_errors_return_before_any_cuda_call():
     assert _fwd(scale=0.0) == fa.FA_ERR_INVALID_ARG
     assert _fwd(scale=float("nan")) == fa.FA_ERR_INVALID_ARG
     assert _fwd(scale=-1.0) == fa.FA_ERR_INVALID_ARG
-    assert _fwd(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(d=80) == fa.FA_ERR_UNSUPPORTED
     assert _fwd(d=32) == fa.FA_ERR_UNSUPPORTED
     # misaligned pointer
     assert fa.lib.fa_fwd(ctypes.c_void_p(18), ctypes.c_void_p(16), ctypes.c_void_p(16),
@@ -109,7 +112,7 @@ def _dec(q=1, k=1, v=1, o=1, lse=None, B=1, Hq=8, Hkv=2, Nq=1, Nk=300, d=128, sc
 
 
 def test_decode_argument_errors_return_before_any_cuda_call():
-    assert _dec(d=96) == 2                              # unsupported head dim
+    assert _dec(d=80) == 2                              # unsupported head dim
     assert _dec(Hq=6, Hkv=4) == 1                       # Hq not a multiple of Hkv
     assert _dec(Hq=64, Hkv=1, Nq=4) == 1                # 256 rows per key/value head
     assert _dec(Nk=0) == 1

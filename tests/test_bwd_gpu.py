@@ -29,6 +29,7 @@ SMALL = [
     (1, 2, 384, 128, True), (2, 1, 700, 128, False),
     (1, 2, 256, 256, True), (1, 1, 330, 256, False),
     (1, 1, 1, 64, True), (1, 1, 50, 128, True),
+    (1, 2, 300, 96, True), (1, 1, 257, 96, False), (1, 1, 200, 192, True), (1, 1, 130, 192, False),
 ]
 
 

@@ -27,6 +27,8 @@ CASES = [
     (1, 2, 2, 5, 5, 64, True),            # Nq == Nk: the ordinary causal forward
     (1, 6, 3, 1, 1, 128, False),          # one key
     (3, 4, 2, 7, 300, 64, False),
+    (1, 8, 2, 2, 1500, 96, True),         # stored head dims on the 128 / 256 kernels
+    (1, 4, 4, 1, 700, 192, True),
 ]
 
 

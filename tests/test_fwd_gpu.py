@@ -23,6 +23,8 @@ SMALL = [
     (1, 3, 384, 128, True), (2, 2, 1000, 128, False), (1, 2, 1000, 128, True),
     (1, 2, 320, 256, True), (1, 2, 520, 256, False),
     (1, 1, 1, 64, True), (1, 1, 77, 128, False),
+    # stored head dims 96 / 192 (run on the 128 / 256 kernels, zero columns past d)
+    (1, 2, 513, 96, True), (2, 2, 300, 96, False), (1, 2, 400, 192, True), (1, 1, 129, 192, False),
 ]
 
 
@@ -90,7 +92,7 @@ def test_fwd_on_side_stream_and_lse_optional(fa):
 
 
 def test_unsupported_head_dim_raises(fa):
-    q = torch.zeros(1, 1, 128, 96, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(1, 1, 128, 80, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(fa.FAError) as ei:
         fa.attention_forward(q, q, q)
     assert ei.value.status == fa.FA_ERR_UNSUPPORTED
