@@ -335,6 +335,7 @@ using FwdD64 = FwdPick<FA_FWD_D64_KIND, 64, false, FA_FWD_D64_EMU>;
 using FwdD128 = FwdPick<FA_FWD_D128_KIND, 128, false, FA_FWD_EMU>;
 using FwdF8D128 = FwdPick<FA_FWD_F8_KIND, 128, true, FA_FWD_F8_EMU>;
 using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_D256_EMU>;
+using FwdF8D256 = FwdCfg<256, 128, 3, 2, true, FA_FWD_F8_EMU>;
 
 #ifndef FA_BWD_EMU
 #define FA_BWD_EMU 1
@@ -595,7 +596,8 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
                      int N, int d, float scale, int causal, void* stream) {
   bool empty = false;
   if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
-  if (d != 128) return fail(FA_ERR_UNSUPPORTED, "FP8 head dim %d not supported (128)", d);
+  if (d != 64 && d != 96 && d != 128 && d != 192 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "FP8 head dim %d not supported (64, 96, 128, 192, 256)", d);
   if (empty) return FA_OK;
   const void* ptrs[] = {q8, k8, v8, o};
   const char* names[] = {"q8", "k8", "v8", "o"};
@@ -618,7 +620,10 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
-  return FwdF8D128::launch(q8, k8, v8, p, static_cast<cudaStream_t>(stream));
+  // d <= 128 on the d = 128 kernel, larger on the one-tile d = 256 kernel (128-key tiles, as
+  // the per-128-row scales need); narrower rows load zero columns past d
+  if (d <= 128) return FwdF8D128::launch(q8, k8, v8, p, static_cast<cudaStream_t>(stream));
+  return launch_fwd<FwdF8D256>(q8, k8, v8, p, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -797,7 +802,14 @@ int fa_version(void) { return 100; }
 
 const char* fa_fwd_kernel_name(int head_dim, int fp8) {
   using namespace fa;
-  if (fp8) return head_dim == 128 ? FwdF8D128::name() : nullptr;
+  if (fp8) {
+    if (head_dim == 64 || head_dim == 96 || head_dim == 128) return FwdF8D128::name();
+    if (head_dim == 192 || head_dim == 256) {
+      static const std::string n = "fa_fwd_kernel<FwdCfg<256,KST3,VST2,e4m3>>";
+      return n.c_str();
+    }
+    return nullptr;
+  }
   switch (head_dim) {
     case 64: return FwdD64::name();
     case 96:

@@ -49,7 +49,9 @@ def test_forward_kernel_names():
     # stored head dims 96 and 192 run on the 128 and 256 kernels
     assert fa.fa_fwd_kernel_name(96) == fa.fa_fwd_kernel_name(128)
     assert fa.fa_fwd_kernel_name(192) == fa.fa_fwd_kernel_name(256)
-    assert fa.fa_fwd_kernel_name(64, True) is None
+    assert fa.fa_fwd_kernel_name(80, True) is None
+    assert fa.fa_fwd_kernel_name(64, True) == fa.fa_fwd_kernel_name(128, True)
+    assert "<256," in fa.fa_fwd_kernel_name(192, True)
 
 
 def _fwd(q=1, k=1, v=1, o=1, lse=None, B=1, H=1, N=128, d=128, scale=0.1, causal=0):
@@ -84,7 +86,7 @@ def test_fp8_and_bwd_argument_errors():
     P = lambda x: ctypes.c_void_p(16 * x)
     st = fa.lib.fa_fwd_fp8(P(1), P(1), P(1), None, P(1), P(1), P(1), None, 1, 1, 256, 128, 0.1, 1, None)
     assert st == fa.FA_ERR_INVALID_ARG
-    st = fa.lib.fa_fwd_fp8(P(1), P(1), P(1), P(1), P(1), P(1), P(1), None, 1, 1, 256, 64, 0.1, 1, None)
+    st = fa.lib.fa_fwd_fp8(P(1), P(1), P(1), P(1), P(1), P(1), P(1), None, 1, 1, 256, 80, 0.1, 1, None)
     assert st == fa.FA_ERR_UNSUPPORTED
     need = fa.fa_bwd_workspace_size(2, 3, 1000, 64)
     assert need >= 2 * 3 * 1000 * 4 and need % 256 == 0

@@ -28,10 +28,15 @@ def dequant(inp):
     return [workloads.dequantize_e4m3_per_tile(inp[n + "8"], inp[n + "s"]) for n in "qkv"]
 
 
-@pytest.mark.parametrize("B,H,N,causal", [(1, 2, 256, True), (2, 2, 640, False),
-                                          (1, 3, 1000, True), (1, 1, 130, False)])
-def test_fp8_small_matches_oracle(fa, B, H, N, causal):
-    w = workloads.make_small(B, H, N, 128, causal, seed=N + 17, backward=False)
+@pytest.mark.parametrize("B,H,N,d,causal", [
+    (1, 2, 256, 128, True), (2, 2, 640, 128, False), (1, 3, 1000, 128, True),
+    (1, 1, 130, 128, False),
+    # narrower and wider heads: 64 and 96 on the 128 kernel, 192 and 256 on the 256 kernel
+    (1, 2, 515, 64, True), (1, 1, 300, 96, False), (1, 2, 700, 256, True),
+    (2, 1, 257, 192, False),
+])
+def test_fp8_small_matches_oracle(fa, B, H, N, d, causal):
+    w = workloads.make_small(B, H, N, d, causal, seed=N + 17 + d, backward=False)
     inp = workloads.make_fp8_inputs(w)
     o, lse = run_fp8(fa, inp, causal, w.sm_scale)
     qd, kd, vd = dequant(inp)
