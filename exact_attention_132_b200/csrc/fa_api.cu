@@ -25,6 +25,11 @@ namespace fa {
 
 // Device status word written by kernels whose bounded waits expired.
 __device__ unsigned g_fa_status = 0;
+// Work counters of the forward kernels' dynamic scheduler, one pair per stream that
+// launched a forward on this device.  A launch leaves its pair at zero when it ends, so
+// launches in one stream (which run one after the other) can share it.
+constexpr int kSchedSlots = 256;
+__device__ int g_fa_sched[kSchedSlots][2];
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 constexpr int kMaxDevices = 64;
@@ -51,6 +56,10 @@ struct DeviceInfo {
   cudaError_t err = cudaSuccess;
   int sms = 0;
   unsigned* status = nullptr;
+  int* sched = nullptr;                 // g_fa_sched of this device
+  std::mutex sched_mu;
+  cudaStream_t sched_stream[kSchedSlots] = {};
+  int sched_used = 0;
 };
 DeviceInfo g_dev[kMaxDevices];
 
@@ -70,10 +79,26 @@ fa_status device_info(DeviceInfo** out) {
     }
     if (d.err == cudaSuccess)
       d.err = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_fa_status);
+    if (d.err == cudaSuccess)
+      d.err = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.sched), g_fa_sched);
   });
   if (d.err != cudaSuccess) return cuda_fail(d.err, "device setup (needs an sm_100 GPU)");
   *out = &d;
   return FA_OK;
+}
+
+// The scheduler counter pair of `stream`.  Streams get slots in order of first use;
+// beyond kSchedSlots distinct streams the slots are reused round-robin, so at most
+// kSchedSlots streams may run forwards on one device at the same time.
+int* sched_counter(DeviceInfo* d, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(d->sched_mu);
+  const int n = d->sched_used < kSchedSlots ? d->sched_used : kSchedSlots;
+  for (int i = 0; i < n; ++i)
+    if (d->sched_stream[i] == stream) return d->sched + 2 * i;
+  const int i = d->sched_used % kSchedSlots;
+  d->sched_stream[i] = stream;
+  ++d->sched_used;
+  return d->sched + 2 * i;
 }
 
 // ------------------------------------------------------------------ tensor maps
@@ -168,6 +193,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, FwdParams p, c
   p.group_heads = causal_group_heads(p.BH, 2ll * p.N * C::D * C::ELEM);
   p.status = di->status;
   p.timeout_ns = kWaitTimeoutNs;
+  p.sched = sched_counter(di, stream);
   const int grid = p.total_items < di->sms ? p.total_items : di->sms;
   kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   cudaError_t e = cudaGetLastError();
@@ -193,7 +219,7 @@ fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p
     cudaFuncAttributes fa_attr;
     cudaError_t e = cudaFuncGetAttributes(&fa_attr, kern);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-    if (fa_attr.numRegs * C::THREADS < 2 * 128 * C::REGS_SOFTMAX + 128 * C::REGS_OTHER)
+    if (fa_attr.numRegs * C::THREADS < C::REGS_TOTAL)
       return fail(FA_ERR_CUDA, "forward kernel built with %d registers/thread: too few for its "
                   "register split", fa_attr.numRegs);
   }
@@ -205,6 +231,7 @@ fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p
   p.group_heads = causal_group_heads(p.BH, 2ll * p.N * C::D * C::ELEM);
   p.status = di->status;
   p.timeout_ns = kWaitTimeoutNs;
+  p.sched = sched_counter(di, stream);
   const int grid = p.total_items < di->sms ? p.total_items : di->sms;
   kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   cudaError_t e = cudaGetLastError();
@@ -236,6 +263,7 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
   p.group_heads = causal_group_heads(p.BH, 2ll * p.N * C::D * C::ELEM);
   p.status = di->status;
   p.timeout_ns = kWaitTimeoutNs;
+  p.sched = sched_counter(di, stream);
   const int grid = p.total_items < di->sms ? p.total_items : di->sms;
   kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   cudaError_t e = cudaGetLastError();
@@ -245,10 +273,11 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 
 // Tuning knobs (compile-time): software-exp2 share, pipeline depth, kernel family.
 // software-exp2 share (quarters of the exponentials) per problem class, measured: the
-// two-tile kernel (d = 64, FP8) gains from 2, the split-softmax d = 128 kernel wants 1,
-// the d = 256 kernel (tensor-core bound) none
+// two-tile kernel gains from 2 at d = 64 and FP8 but wants none at bf16 d = 128 (its
+// per-step path is issue-bound there, not bound by the special-function unit); the
+// d = 256 kernel (tensor-core bound) none
 #ifndef FA_FWD_EMU
-#define FA_FWD_EMU 1
+#define FA_FWD_EMU 0
 #endif
 #ifndef FA_FWD_D64_EMU
 #define FA_FWD_D64_EMU 2
@@ -290,7 +319,7 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #define FA_FWD_D64_KIND 1
 #endif
 #ifndef FA_FWD_D128_KIND
-#define FA_FWD_D128_KIND 2
+#define FA_FWD_D128_KIND 1
 #endif
 #ifndef FA_FWD_F8_KIND
 #define FA_FWD_F8_KIND 1

@@ -58,6 +58,7 @@ struct FwdParams {
   const float* v_scale;
   unsigned* status;
   unsigned long long timeout_ns;
+  int* sched;         // {next item, CTAs finished}: zero at launch, zero again at exit
 };
 
 // Key/value head of query head `bh` (flattened b * H + h): K/V hold H / g heads per
@@ -121,6 +122,68 @@ struct FwdCfg {
 __device__ __forceinline__ int fwd_item_index(int k) {
   const int pos = (k & 1) ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
   return k * gridDim.x + pos;
+}
+
+// ---------------------------------------------------------------- dynamic work distribution
+// A CTA's first item is blockIdx.x; each further one is drawn by the producer thread
+// from a global counter, so a CTA that finishes early takes the next item and the
+// heaviest-first causal order balances itself (a static round-robin of the same order
+// leaves the CTAs that drew the longest rows working alone at the end).  The producer
+// publishes every item in a small shared-memory ring that the other roles read; a value
+// >= total_items ends every role's loop.  The last CTA to leave sets the counter back to
+// zero for the next launch on the same stream.
+constexpr int kItemSlots = 4;
+constexpr int kItemBytes = 2 * kItemSlots * 8 + kItemSlots * 4;   // barriers, then slots
+
+struct ItemRing {
+  uint32_t bars;        // kItemSlots "full" barriers, then kItemSlots "empty" barriers
+  volatile int* slot;   // kItemSlots item values
+  // one-time setup by a single thread: `readers` arrivals release a slot
+  __device__ __forceinline__ void init(uint32_t readers) const {
+    for (int s = 0; s < kItemSlots; ++s) {
+      mbar_init(bars + 8u * s, 1u);
+      mbar_init(bars + 8u * (kItemSlots + s), readers);
+    }
+  }
+  // producer thread: draw item k and publish it; false when a wait gave up
+  __device__ __forceinline__ bool put(const FwdParams& p, int k, int& w, const WaitCtl& wc) const {
+    w = k == 0 ? static_cast<int>(blockIdx.x) : static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1);
+    const int s = k % kItemSlots;
+    if (k >= kItemSlots &&
+        !mbar_wait(bars + 8u * (kItemSlots + s), ((k / kItemSlots) - 1) & 1, wc, kSiteItem))
+      return false;
+    slot[s] = w;
+    mbar_arrive(bars + 8u * s);   // release: the slot value is visible to every waiter
+    return true;
+  }
+  // one reader thread: read item k and release its slot
+  __device__ __forceinline__ bool get(int k, int& w, const WaitCtl& wc) const {
+    const int s = k % kItemSlots;
+    if (!mbar_wait(bars + 8u * s, (k / kItemSlots) & 1, wc, kSiteItem)) return false;
+    w = slot[s];
+    mbar_arrive(bars + 8u * (kItemSlots + s));
+    return true;
+  }
+  // every lane of a warp reads item k; the warp releases the slot once
+  __device__ __forceinline__ bool get_warp(int k, int& w, const WaitCtl& wc) const {
+    const int s = k % kItemSlots;
+    if (!mbar_wait_warp(bars + 8u * s, (k / kItemSlots) & 1, wc, kSiteItem)) return false;
+    w = slot[s];
+    mbar_arrive_warp(bars + 8u * (kItemSlots + s));
+    return true;
+  }
+};
+
+// Thread 0 of each CTA after every role has left its item loop: the last CTA out
+// resets the counter.  Every draw of a CTA completes (its value is used) before that
+// CTA's arrival here, so the reset follows the final draw of the launch.
+__device__ __forceinline__ void sched_release(const FwdParams& p) {
+  __threadfence();
+  if (atomicAdd(p.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+    p.sched[0] = 0;
+    p.sched[1] = 0;
+    __threadfence();
+  }
 }
 
 // Map a linear item to (bh, q tile).  Non-causal: head-major, so CTAs running at

@@ -58,7 +58,9 @@ struct PPCfg {
                        B_DRAIN = 10, B_KFULL = 11, B_KEMPTY = 11 + KST, B_VFULL = 11 + 2 * KST,
                        B_VEMPTY = 11 + 2 * KST + VST, NBARS = 11 + 2 * KST + 2 * VST;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
-  static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
+  static constexpr int SMEM_ITEM = SMEM_MISC + 64;    // work-item ring
+  static constexpr int SMEM_ALLOC = SMEM_ITEM + kItemBytes + 1024;
+  static constexpr uint32_t ITEM_READERS = 1 + 8;     // the MMA thread and 8 softmax warps
   static constexpr int TM_S = 0;                     // + t * BN
   static constexpr int TM_O = 2 * BN;                // + t * D
   static constexpr int TM_COLS = 512;
@@ -69,7 +71,8 @@ struct PPCfg {
   static constexpr int THREADS = 384;
   static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
   static constexpr int REGS_SOFTMAX = 208, REGS_OTHER = 88;
-  static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * 168, "register split");
+  static constexpr int REGS_TOTAL = 2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER;
+  static_assert(REGS_TOTAL <= THREADS * 168, "register split");
   static_assert(2 * BN + 2 * D <= TM_COLS, "tensor memory budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
@@ -123,7 +126,8 @@ __device__ __forceinline__ void pp_issue_pv(uint32_t o_tmem, uint32_t p_tmem, ui
 // reload them.
 template <class C>
 __device__ void pp_producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
-                            const FwdParams& p, uint32_t sbase, uint32_t bars, const WaitCtl& wc) {
+                            const FwdParams& p, uint32_t sbase, uint32_t bars, const ItemRing& ring,
+                            const WaitCtl& wc) {
   const uint32_t b_qfull0 = bars + 8u * C::B_QFULL, b_qfull1 = b_qfull0 + 8u;
   const uint32_t b_qempty0 = bars + 8u * C::B_QEMPTY, b_qempty1 = b_qempty0 + 8u;
   const uint32_t b_kfull = bars + 8u * C::B_KFULL, b_kempty = bars + 8u * C::B_KEMPTY;
@@ -131,7 +135,8 @@ __device__ void pp_producer(const CUtensorMap* tq, const CUtensorMap* tk, const 
   uint32_t gk = 0, gv = 0, tq0 = 0, tq1 = 0;
   bool ok = true;
   for (int k = 0; ok; ++k) {
-    const int w = fwd_item_index(k);
+    int w;
+    if (!(ok = ring.put(p, k, w, wc))) break;
     if (w >= p.total_items) break;
     int bh, pr;
     pp_decode_item(p, w, bh, pr);
@@ -207,7 +212,7 @@ __device__ void pp_producer(const CUtensorMap* tq, const CUtensorMap* tk, const 
 // ---------------------------------------------------------------- MMA issuer (one thread)
 template <class C>
 __device__ void pp_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
-                       const WaitCtl& wc) {
+                       const ItemRing& ring, const WaitCtl& wc) {
   const uint32_t b_qfull0 = bars + 8u * C::B_QFULL, b_qfull1 = b_qfull0 + 8u;
   const uint32_t b_qempty0 = bars + 8u * C::B_QEMPTY, b_qempty1 = b_qempty0 + 8u;
   const uint32_t b_sfull0 = bars + 8u * C::B_SFULL, b_sfull1 = b_sfull0 + 8u;
@@ -226,7 +231,8 @@ __device__ void pp_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32
   uint32_t g = 0, gs0 = 0, gs1 = 0, tq0 = 0, tq1 = 0;
   bool ok = true;
   for (int k = 0; ok; ++k) {
-    const int w = fwd_item_index(k);
+    int w;
+    if (!(ok = ring.get(k, w, wc))) break;
     if (w >= p.total_items) break;
     int bh, pr;
     pp_decode_item(p, w, bh, pr);
@@ -295,7 +301,8 @@ __device__ void pp_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32
 
 // ---------------------------------------------------------------- softmax (one tile)
 template <class C>
-__device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int t, const WaitCtl& wc) {
+__device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int t, const ItemRing& ring,
+                           const WaitCtl& wc) {
   auto bar = [&](int i) { return bars + 8u * i; };
   const int warp = threadIdx.x / 32;
   const int quad = warp & 3;
@@ -310,7 +317,8 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
   bool ok = true;
 
   for (int k = 0; ok; ++k) {
-    const int w = fwd_item_index(k);
+    int w;
+    if (!(ok = ring.get_warp(k, w, wc))) break;
     if (w >= p.total_items) break;
     int bh, pr;
     pp_decode_item(p, w, bh, pr);
@@ -504,11 +512,11 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       ++gs;
     }
     if (!ok) break;
+    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / l;
+    const bool row_ok = q_idx < p.N;
     if (!(ok = mbar_wait(bar(C::B_ODONE + t), ti & 1, wc, kSiteODone))) break;
     ++ti;
     tc_fence_after();
-    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / l;
-    const bool row_ok = q_idx < p.N;
     __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * p.ld;
 #pragma unroll 1
     for (int c = 0; c < C::D; c += 32) {
@@ -543,11 +551,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const uint32_t bars = sbase + C::SMEM_BAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
+  const ItemRing ring{sbase + C::SMEM_ITEM,
+                      reinterpret_cast<volatile int*>(smem + C::SMEM_ITEM + 2 * kItemSlots * 8)};
   const int warp = threadIdx.x / 32;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i)
       mbar_init(bars + 8u * i, (i == C::B_PFULL || i == C::B_PFULL + 1) ? 4u : 1u);  // warps
+    ring.init(C::ITEM_READERS);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tq);
@@ -567,16 +578,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (warp >= 8) {
     regs_decrease<C::REGS_OTHER>();
     if (warp == C::PRODUCER_WARP && (threadIdx.x & 31) == 0)
-      pp_producer<C>(&tq, &tk, &tv, p, sbase, bars, wc);
+      pp_producer<C>(&tq, &tk, &tv, p, sbase, bars, ring, wc);
     else if (warp == C::MMA_WARP && (threadIdx.x & 31) == 0)
-      pp_mma<C>(p, sbase, bars, tmem, wc);
+      pp_mma<C>(p, sbase, bars, tmem, ring, wc);
   } else {
     regs_increase<C::REGS_SOFTMAX>();
-    pp_softmax<C>(p, bars, tmem, warp / 4, wc);
+    pp_softmax<C>(p, bars, tmem, warp / 4, ring, wc);
   }
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) sched_release(p);
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);

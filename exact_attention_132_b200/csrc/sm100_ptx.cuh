@@ -18,7 +18,8 @@ constexpr unsigned kStatusTimeout = 4u << 24;
 
 enum WaitSite : unsigned {
   kSiteQFull = 1, kSiteQEmpty, kSiteKFull, kSiteVFull, kSiteKVEmpty, kSiteSFull, kSitePFull,
-  kSiteODone, kSiteDrain, kSiteDsFull, kSiteDqDone, kSiteXchg, kSitePvDone, kSiteSelfTest = 99
+  kSiteODone, kSiteDrain, kSiteDsFull, kSiteDqDone, kSiteXchg, kSitePvDone, kSiteItem,
+  kSiteSelfTest = 99
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
