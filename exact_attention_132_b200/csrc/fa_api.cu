@@ -420,6 +420,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     BwdParams pk = p;
     pk.n_qt = (p.N + CK::BMQ - 1) / CK::BMQ;
     pk.n_kt = (p.N + CK::BN - 1) / CK::BN;
+    // a K/V head streams its g query heads' Q and dO
+    pk.group_heads = causal_group_heads(p.BH / p.g, 4ll * p.g * p.N * p.ld);
     // one CTA per key/value head, key tile and d part
     const long long grid = static_cast<long long>(p.BH / p.g) * pk.n_kt * CK::NSPLIT;
     kern<<<static_cast<unsigned>(grid), CK::THREADS, CK::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, pk);
@@ -438,6 +440,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     BwdParams pq = p;
     pq.n_qt = (p.N + CQ::BM - 1) / CQ::BM;
     pq.n_kt = (p.N + CQ::BN - 1) / CQ::BN;
+    pq.group_heads = causal_group_heads(p.BH, 4ll * p.N * p.ld);   // K and V of the head
     const long long grid = static_cast<long long>(p.BH) * pq.n_qt;
     kern<<<static_cast<unsigned>(grid), CQ::THREADS, CQ::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, pq);
     cudaError_t e = cudaGetLastError();

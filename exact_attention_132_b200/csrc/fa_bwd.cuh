@@ -39,6 +39,7 @@ struct BwdParams {
   int n_qt;              // query tiles of BMQ rows (dK/dV pass) / 128 rows (dQ pass)
   int n_kt;              // key tiles
   int causal;
+  int group_heads;       // heads per level-major sweep of the CTA order (bwd_block_item)
   float scale;
   const float* lse;      // [BH, N]
   const float* drow;     // D_i workspace [BH, N]
@@ -48,6 +49,24 @@ struct BwdParams {
   unsigned* status;
   unsigned long long timeout_ns;
 };
+
+// CTA -> (head, level, part).  Heads go in groups of p.group_heads; inside a group the
+// order is level-major: level 0 (the heaviest causal tile) of every head of the group,
+// then level 1, ...  The hardware hands out CTAs in index order, so the long tiles
+// start first and the short ones fill the end (a head-major order leaves the last
+// heads' long tiles running alone), while the CTAs in flight together stream only one
+// group's operands through L2.
+__device__ __forceinline__ void bwd_block_item(int block, int heads, int levels, int parts,
+                                               int group, int& head, int& lvl, int& part) {
+  part = block % parts;
+  int r = block / parts;
+  const int per_group = group * levels;
+  const int gi = r / per_group;
+  r -= gi * per_group;
+  const int gsize = min(group, heads - gi * group);
+  lvl = r / gsize;
+  head = gi * group + (r - lvl * gsize);
+}
 
 // --------------------------------------------------------------------------- 1. D_i
 // D_i = sum_c dO_ic * O_ic, fp32 accumulation of the bf16 products.  A row of D
@@ -217,10 +236,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // block -> (key/value head, key tile, d part); heaviest causal tiles (small kt) first.
   // With grouped heads the g query heads reading this K/V head all contribute to its
   // dK, dV: the steps run over (query head of the group, query tile).
-  const int split = blockIdx.x % C::NSPLIT;
-  const int rest = blockIdx.x / C::NSPLIT;
-  const int kt = rest % p.n_kt;
-  const int bh = rest / p.n_kt;                       // key/value head (b * H / g + h / g)
+  int split, kt, bh;                                  // bh: key/value head (b * H / g + h / g)
+  bwd_block_item(blockIdx.x, p.BH / p.g, p.n_kt, C::NSPLIT, p.group_heads, bh, kt, split);
   int i0, i1;
   dkdv_q_range<C>(p, kt, i0, i1);
   const int nqt = i1 - i0;                            // query tiles per query head
@@ -598,9 +615,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
 
   // block -> (bh, q tile); highest causal q tile (most key tiles) first
-  const int bh = blockIdx.x / p.n_qt;
+  int bh, lvl, part;
+  bwd_block_item(blockIdx.x, p.BH, p.n_qt, 1, p.group_heads, bh, lvl, part);
   const int bkv = p.g == 1 ? bh : (bh / p.H) * (p.H / p.g) + (bh % p.H) / p.g;   // K/V head
-  const int qt = p.n_qt - 1 - (blockIdx.x - bh * p.n_qt);
+  const int qt = p.n_qt - 1 - lvl;
   const int nsteps = p.causal ? min(p.n_kt, ((qt + 1) * C::BM - 1) / C::BN + 1) : p.n_kt;
 
   if (threadIdx.x == 0) {
