@@ -46,8 +46,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # fa_fwd_d128_causal_B4H16N4096.md), keyed by a hash of the kernel sources and the
 # launched kernel's name (which carries its tile configuration).  A changed kernel has
 # no entry and reports traffic = null.
-FWD_TRAFFIC_BYTES = {"cd33a9aede1cbebf": 269_234_176}
+FWD_TRAFFIC_BYTES = {"458f58bcb3cccb4b": 248_615_424}
 KERNEL_SOURCES = ("exact_attention_132_b200/csrc/fa_fwd.cuh",
+                  "exact_attention_132_b200/csrc/fa_fwd_pp.cuh",
                   "exact_attention_132_b200/csrc/fa_fwd_ws.cuh",
                   "exact_attention_132_b200/csrc/sm100_ptx.cuh")
 
