@@ -61,6 +61,10 @@ struct FwdParams {
   int* sched;         // {next item, CTAs finished}: zero at launch, zero again at exit
 };
 
+// Shared-memory ring of work items (ItemRing below): slots and bytes
+constexpr int kItemSlots = 4;
+constexpr int kItemBytes = 2 * kItemSlots * 8 + kItemSlots * 4;   // barriers, then slots
+
 // Key/value head of query head `bh` (flattened b * H + h): K/V hold H / g heads per
 // batch entry and query head h reads K/V head h / g.
 __device__ __forceinline__ int fwd_kv_head(const FwdParams& p, int bh) {
@@ -104,7 +108,9 @@ struct FwdCfg {
                        B_DRAIN = 7, B_KFULL = 8, B_KEMPTY = 8 + KST, B_VFULL = 8 + 2 * KST,
                        B_VEMPTY = 8 + 2 * KST + VST, NBARS = 8 + 2 * KST + 2 * VST;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;   // tmem slot, abort flag, reductions
-  static constexpr int SMEM_TOTAL = SMEM_MISC + 64;
+  static constexpr int SMEM_ITEM = SMEM_MISC + 64;         // work-item ring
+  static constexpr int SMEM_TOTAL = SMEM_ITEM + kItemBytes;
+  static constexpr uint32_t ITEM_READERS = 1 + 4;          // the MMA thread, 4 softmax warps
   static constexpr int SMEM_ALLOC = SMEM_TOTAL + 1024;     // slack to align the base to 1024
   static constexpr int TM_S = 0;
   static constexpr int TM_O = 2 * BN;
@@ -132,9 +138,6 @@ __device__ __forceinline__ int fwd_item_index(int k) {
 // publishes every item in a small shared-memory ring that the other roles read; a value
 // >= total_items ends every role's loop.  The last CTA to leave sets the counter back to
 // zero for the next launch on the same stream.
-constexpr int kItemSlots = 4;
-constexpr int kItemBytes = 2 * kItemSlots * 8 + kItemSlots * 4;   // barriers, then slots
-
 struct ItemRing {
   uint32_t bars;        // kItemSlots "full" barriers, then kItemSlots "empty" barriers
   volatile int* slot;   // kItemSlots item values
@@ -214,7 +217,8 @@ __device__ __forceinline__ int fwd_num_kv_tiles(const FwdParams& p, int qt) {
 // ---------------------------------------------------------------- producer (one thread)
 template <class C>
 __device__ void fwd_producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
-                             const FwdParams& p, uint32_t sbase, uint32_t bars, const WaitCtl& wc) {
+                             const FwdParams& p, uint32_t sbase, uint32_t bars, const ItemRing& ring,
+                             const WaitCtl& wc) {
   auto bar = [&](int i) { return bars + 8u * i; };
   // Loads follow the order the MMA warp consumes them: per item Q, K_0, then
   // (K_j, V_{j-1}) for j >= 1, then V_{n-1}; K therefore runs one step ahead of V.
@@ -245,7 +249,8 @@ __device__ void fwd_producer(const CUtensorMap* tq, const CUtensorMap* tk, const
     return true;
   };
   for (int k = 0; ok; ++k) {
-    const int w = fwd_item_index(k);
+    int w;
+    if (!(ok = ring.put(p, k, w, wc))) break;
     if (w >= p.total_items) break;
     int bh, qt;
     fwd_decode_item(p, w, bh, qt);
@@ -285,7 +290,7 @@ __device__ void fwd_producer(const CUtensorMap* tq, const CUtensorMap* tk, const
 // ---------------------------------------------------------------- MMA issuer (one thread)
 template <class C>
 __device__ void fwd_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
-                        const WaitCtl& wc) {
+                        const ItemRing& ring, const WaitCtl& wc) {
   auto bar = [&](int i) { return bars + 8u * i; };
   constexpr uint32_t IDESC_S = C::FP8 ? idesc_e4m3(128, C::BN, false) : idesc_bf16(128, C::BN, false);
   constexpr uint32_t IDESC_O = C::FP8 ? idesc_e4m3(128, C::D, true) : idesc_bf16(128, C::D, true);
@@ -316,7 +321,8 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t sbase, uint32_t bars, uint3
   };
 
   for (int k = 0; ok; ++k) {
-    const int w = fwd_item_index(k);
+    int w;
+    if (!(ok = ring.get(k, w, wc))) break;
     if (w >= p.total_items) break;
     int bh, qt;
     fwd_decode_item(p, w, bh, qt);
@@ -378,7 +384,8 @@ __device__ __forceinline__ uint64_t ex2_f16_pair(uint64_t x2) {
 
 // ---------------------------------------------------------------- softmax warps
 template <class C>
-__device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, const WaitCtl& wc) {
+__device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, const ItemRing& ring,
+                            const WaitCtl& wc) {
   auto bar = [&](int i) { return bars + 8u * i; };
   const int warp = threadIdx.x / 32;
   const int quad = warp & 3;
@@ -392,7 +399,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
   bool ok = true;
 
   for (int k = 0; ok; ++k) {
-    const int w = fwd_item_index(k);
+    int w;
+    if (!(ok = ring.get_warp(k, w, wc))) break;
     if (w >= p.total_items) break;
     int bh, qt;
     fwd_decode_item(p, w, bh, qt);
@@ -573,6 +581,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const uint32_t bars = sbase + C::SMEM_BAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
+  const ItemRing ring{sbase + C::SMEM_ITEM,
+                      reinterpret_cast<volatile int*>(smem + C::SMEM_ITEM + 2 * kItemSlots * 8)};
   const int warp = threadIdx.x / 32;
 
   if (threadIdx.x == 0) {
@@ -581,6 +591,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (i == C::B_PFULL || i == C::B_PFULL + 1) cnt = 4;   // one arrival per softmax warp
       mbar_init(bars + 8u * i, cnt);
     }
+    ring.init(C::ITEM_READERS);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tq);
@@ -598,15 +609,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const WaitCtl wc{abort_flag, p.status, p.timeout_ns};
 
   if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) fwd_producer<C>(&tq, &tk, &tv, p, sbase, bars, wc);
+    if ((threadIdx.x & 31) == 0) fwd_producer<C>(&tq, &tk, &tv, p, sbase, bars, ring, wc);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) fwd_mma<C>(p, sbase, bars, tmem, wc);
+    if ((threadIdx.x & 31) == 0) fwd_mma<C>(p, sbase, bars, tmem, ring, wc);
   } else {
-    fwd_softmax<C>(p, bars, tmem, wc);
+    fwd_softmax<C>(p, bars, tmem, ring, wc);
   }
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) sched_release(p);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
