@@ -360,6 +360,21 @@ def run_extras(fa, dev, stream, steps, peak, hbm_peak):
                        "ms_fwd": round(tot / steps, 3),
                        "frac_of_fp8_nominal_2x_bf16_peak":
                            round(w.fwd_flops() * steps / (tot * 1e-3) / 1e12 / (2 * peak), 4)}
+    # FP8 backward on the same inputs: dequantisation passes + the bf16 backward
+    gen.manual_seed(w.seed + 1)
+    do = torch.randn(shp, generator=gen, device=dev).to(torch.bfloat16)
+    dq, dk, dv = (torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(3))
+    ws = torch.empty(max(1, fa.fa_bwd_fp8_workspace_size(*shp)), dtype=torch.uint8, device=dev)
+    f8()
+    b8 = lambda: fa.fa_bwd_fp8(t8["q"], t8["k"], t8["v"], sc["q"], sc["k"], sc["v"], o, do, lse,
+                               dq, dk, dv, ws, scale=w.sm_scale, causal=True, stream=stream)
+    bsteps = max(3, steps // 3)
+    btot, _ = time_steps(b8, bsteps, 1, stream)
+    out["fp8_d128"].update({
+        "tflops_bwd": round(w.bwd_flops() * bsteps / (btot * 1e-3) / 1e12, 2),
+        "ms_bwd": round(btot / bsteps, 3),
+        "bwd_note": "gradients for the dequantised inputs: e4m3 -> bf16 pass, then the bf16 "
+                    "backward (metric FLOPs 2.5x the forward's)"})
     return out
 
 

@@ -64,6 +64,10 @@ def _load() -> ctypes.CDLL:
     L.fa_decode.restype = ctypes.c_int
     L.fa_fwd_kernel_name.argtypes = [i, i]
     L.fa_fwd_kernel_name.restype = ctypes.c_char_p
+    L.fa_bwd_fp8_workspace_size.argtypes = [i, i, i, i]
+    L.fa_bwd_fp8_workspace_size.restype = sz
+    L.fa_bwd_fp8.argtypes = [vp] * 13 + [sz, i, i, i, i, f, i, vp]
+    L.fa_bwd_fp8.restype = ctypes.c_int
     for name in ("fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_get_device_status",
                  "fa_debug_wait_timeout_selftest", "fa_version"):
         getattr(L, name).restype = ctypes.c_int
@@ -232,6 +236,49 @@ def attention_backward(q, k, v, o, dO, lse, causal: bool = False, scale: float |
         nbytes = fa_bwd_workspace_size(B, H, N, d)
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
     fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, scale=scale, causal=causal)
+    return dq, dk, dv
+
+
+def fa_bwd_fp8_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib.fa_bwd_fp8_workspace_size(B, H, N, d))
+
+
+def fa_bwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, dO, lse, dq, dk, dv, workspace,
+               scale: float | None = None, causal: bool = False, stream=None):
+    """Gradients (bf16) for the dequantised inputs of the FP8 forward: o and lse are
+    fa_fwd_fp8's outputs; the workspace holds bf16 copies of q8, k8, v8 times their tile
+    scales and the row sums of the backward."""
+    B, H, N, d = _bhnd(q8, "q8", torch.float8_e4m3fn)
+    for t, n in ((k8, "k8"), (v8, "v8")):
+        if _bhnd(t, n, torch.float8_e4m3fn) != (B, H, N, d):
+            raise ValueError(f"{n} shape differs from q8")
+    for t, n in ((o, "o"), (dO, "dO"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if _bhnd(t, n, torch.bfloat16) != (B, H, N, d):
+            raise ValueError(f"{n} shape differs from q8")
+    nt = (N + 127) // 128
+    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        if tuple(t.shape) != (B, H, nt) or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous fp32 [B, H, ceil(N/128)]")
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be fp32 [B, H, N]")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.fa_bwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale),
+                          _ptr(v_scale), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk),
+                          _ptr(dv), _ptr(workspace), ws_bytes, B, H, N, d, sc,
+                          1 if causal else 0, _stream(stream)))
+
+
+def attention_backward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, dO, lse,
+                           causal: bool = False, scale: float | None = None):
+    """Allocate dQ/dK/dV and the workspace and run fa_bwd_fp8."""
+    B, H, N, d = q8.shape
+    dq, dk, dv = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+                  for _ in range(3))
+    nbytes = fa_bwd_fp8_workspace_size(B, H, N, d)
+    workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q8.device)
+    fa_bwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, dO, lse, dq, dk, dv, workspace,
+               scale=scale, causal=causal)
     return dq, dk, dv
 
 

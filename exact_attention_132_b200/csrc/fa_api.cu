@@ -19,6 +19,7 @@
 #include "fa_fwd_ws.cuh"
 #include "fa_fwd_sp.cuh"
 #include "fa_decode.cuh"
+#include "fa_dequant.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa {
@@ -469,6 +470,11 @@ size_t workspace_bytes(int B, int H, int N) {
   return (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
 }
 
+// FP8 backward: one bf16 [B,H,N,d] copy of a dequantised input, 256-byte aligned
+size_t fp8_bwd_tensor_bytes(int B, int H, int N, int d) {
+  return (static_cast<size_t>(B) * H * N * d * 2 + 255) & ~static_cast<size_t>(255);
+}
+
 // ------------------------------------------------------------------ no-allocation backward
 // Fixed scratch for fa_bwd_noalloc: one fp32 D_i per row (B*H*N rows at most
 // FA_BWD_NOALLOC_MAX_ROWS).  It lives in the module image, so every GPU that loads
@@ -709,6 +715,61 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* stream) {
   return fa_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes_, B, H,
                     H > 0 ? H : 1, N, d, scale, causal, stream);
+}
+
+// ------------------------------------------------------------------ FP8 backward
+size_t fa_bwd_fp8_workspace_size(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  return 3 * fp8_bwd_tensor_bytes(B, H, N, d) + workspace_bytes(B, H, N);
+}
+
+fa_status fa_bwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,
+                     const float* k_scale, const float* v_scale, const void* o, const void* dO,
+                     const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                     size_t workspace_bytes_, int B, int H, int N, int d, float scale, int causal,
+                     void* stream) {
+  bool empty = false;
+  if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
+  if (d != 64 && d != 96 && d != 128 && d != 192 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "FP8 head dim %d not supported (64, 96, 128, 192, 256)", d);
+  if (empty) return FA_OK;
+  const void* ptrs[] = {q8, k8, v8, o, dO, lse, dq, dk, dv, workspace};
+  const char* names[] = {"q8", "k8", "v8", "o", "dO", "lse", "dq", "dk", "dv", "workspace"};
+  if (fa_status s = check_ptrs(ptrs, names, 10)) return s;
+  if (!q_scale || !k_scale || !v_scale) return fail(FA_ERR_INVALID_ARG, "FP8 scale pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale) |
+       reinterpret_cast<uintptr_t>(v_scale)) & 3u)
+    return fail(FA_ERR_INVALID_ARG, "FP8 scales must be 4-byte aligned");
+  const size_t need = fa_bwd_fp8_workspace_size(B, H, N, d);
+  if (workspace_bytes_ < need)
+    return fail(FA_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes_, need);
+  DeviceInfo* di = nullptr;
+  if (fa_status s = device_info(&di)) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // 1. the dequantised inputs, bf16, at the front of the workspace
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t tb = fp8_bwd_tensor_bytes(B, H, N, d);
+  void* qd = ws;
+  void* kd = ws + tb;
+  void* vd = ws + 2 * tb;
+  const long long groups = static_cast<long long>(B) * H * N * d / 16;
+  const int n_st = (N + 127) / 128;
+  long long blocks = (groups + 255) / 256;
+  const long long cap = static_cast<long long>(di->sms) * 8;
+  if (blocks > cap) blocks = cap;
+  const void* src[3] = {q8, k8, v8};
+  const float* scl[3] = {q_scale, k_scale, v_scale};
+  void* dst[3] = {qd, kd, vd};
+  for (int t = 0; t < 3; ++t) {
+    fa_dequant_e4m3<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint8_t*>(src[t]), scl[t], static_cast<__nv_bfloat16*>(dst[t]), groups, d,
+        N, n_st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dequantisation kernel launch");
+  }
+  // 2. the bf16 backward on them, with the rest of the workspace for D_i
+  return fa_bwd(qd, kd, vd, o, dO, lse, dq, dk, dv, ws + 3 * tb, need - 3 * tb, B, H, N, d, scale,
+                causal, stream);
 }
 
 // Same kernels and results as fa_bwd, but the per-row D_i scratch comes from the

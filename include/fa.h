@@ -71,7 +71,8 @@ typedef enum {
  *                                  (the normalisation statistic the backward reuses;
  *                                  issoh.co.jp page, section 逆伝播でL×L行列を保存せず
  *                                  再計算する設計).  May be NULL if not wanted.
- * Returns FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED (d not 64/128/256) or FA_ERR_CUDA.
+ * Returns FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED (d not 64/96/128/192/256) or
+ * FA_ERR_CUDA.
  */
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                  int B, int H, int N, int d, float scale, int causal, void* stream);
@@ -86,7 +87,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  *   o                 out bf16 [B,H,N,d]; lse out fp32 [B,H,N] (may be NULL)
  * The probabilities are rounded to e4m3 before the P V product (the product runs
  * on the FP8 tensor cores); everything else accumulates in fp32.
- * d must be 128.  Errors as fa_fwd.
+ * d is 64, 96, 128, 192 or 256.  Errors as fa_fwd.
  */
 fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
                      const float* q_scale, const float* k_scale, const float* v_scale,
@@ -120,6 +121,36 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  const float* lse, void* dq, void* dk, void* dv,
                  void* workspace, size_t workspace_bytes,
                  int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
+ * fa_bwd_fp8_workspace_size — bytes of device workspace fa_bwd_fp8 needs: bf16 copies of
+ * the three dequantised inputs followed by fa_bwd's workspace, each part 256-byte
+ * aligned.  0 when B*H*N*d == 0.
+ */
+size_t fa_bwd_fp8_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_bwd_fp8 — backward of the FP8 forward.  The pages define no FP8 backward; they
+ * note only that FA3 still lacks one (issoh.co.jp page, sections
+ * FA3のhopper配下からの導入とFA4のパッケージ導入 and FlashAttention-3と4のどちらを入れれば
+ * よいですか？).  Reading taken: the gradients of L = sum(O * dO) with respect to the
+ * dequantised inputs Q = q8 * q_scale, K = k8 * k_scale, V = v8 * v_scale (the
+ * quantisation passes gradients straight through), computed by the bf16 backward after
+ * one streaming pass that writes those inputs, rounded to bf16, into the workspace.
+ *   q8, k8, v8, q_scale, k_scale, v_scale   in  as fa_fwd_fp8
+ *   o, lse           in   fa_fwd_fp8's outputs for the same inputs
+ *   dO               in   bf16 [B,H,N,d]
+ *   dq, dk, dv       out  bf16 [B,H,N,d]: gradients for the dequantised Q, K, V
+ *   workspace        scratch device memory of >= fa_bwd_fp8_workspace_size() bytes,
+ *                    owned by the caller; contents on entry are ignored.
+ * Launches, in stream order: three dequantisation passes, then fa_bwd's three passes.
+ * Errors as fa_bwd.
+ */
+fa_status fa_bwd_fp8(const void* q8, const void* k8, const void* v8,
+                     const float* q_scale, const float* k_scale, const float* v_scale,
+                     const void* o, const void* dO, const float* lse,
+                     void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                     int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
  * fa_bwd_noalloc — fa_bwd for callers that cannot allocate device memory.

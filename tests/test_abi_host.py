@@ -95,6 +95,23 @@ def test_fp8_and_bwd_argument_errors():
     assert st == fa.FA_ERR_INVALID_ARG and "workspace" in fa.fa_last_error_string()
 
 
+def test_fp8_bwd_argument_errors():
+    P = lambda x: ctypes.c_void_p(16 * x)
+    need = fa.fa_bwd_fp8_workspace_size(1, 2, 300, 128)
+    # three bf16 copies of the inputs plus the D_i rows, each 256-byte aligned
+    assert need >= 3 * 2 * 300 * 128 * 2 + 2 * 300 * 4 and need % 256 == 0
+    assert fa.fa_bwd_fp8_workspace_size(0, 2, 300, 128) == 0
+    args = [P(1)] * 13
+    st = fa.lib.fa_bwd_fp8(*args, need, 1, 2, 300, 80, 0.1, 1, None)
+    assert st == fa.FA_ERR_UNSUPPORTED
+    st = fa.lib.fa_bwd_fp8(*args, need - 256, 1, 2, 300, 128, 0.1, 1, None)
+    assert st == fa.FA_ERR_INVALID_ARG and "workspace" in fa.fa_last_error_string()
+    no_scale = args[:3] + [None] + args[4:]
+    st = fa.lib.fa_bwd_fp8(*no_scale, need, 1, 2, 300, 128, 0.1, 1, None)
+    assert st == fa.FA_ERR_INVALID_ARG and "scale" in fa.fa_last_error_string()
+    assert fa.lib.fa_bwd_fp8(*([None] * 13), 0, 1, 2, 0, 128, 0.1, 1, None) == fa.FA_OK
+
+
 def test_python_wrappers_validate_shapes():
     import torch
     q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
