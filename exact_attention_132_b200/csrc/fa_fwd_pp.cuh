@@ -23,7 +23,8 @@
 
 namespace fa {
 
-template <int D_, int KST_, int VST_, bool FP8_, int EMU_ = 1, int TAU_ = 0, bool EXPH_ = false>
+template <int D_, int KST_, int VST_, bool FP8_, int EMU_ = 1, int TAU_ = 0, bool EXPH_ = false,
+          bool COMP_ = false>
 struct PPCfg {
   static constexpr int D = D_;
   static constexpr int BN = 128;
@@ -41,6 +42,13 @@ struct PPCfg {
   // bf16 only: exponentials on the special-function unit in half precision, two
   // values per instruction (ex2.approx.f16x2).
   static constexpr bool EXPH = EXPH_ && !FP8;
+  // TAU > 0 without the per-element rounded sum: the row sum adds the unrounded
+  // probabilities plus, per key tile, the bf16 rounding error of the tile's largest
+  // probability (the one that may exceed 1 and dominate the row).  The P V product
+  // uses every probability rounded; only the largest one's error is large enough to
+  // bias O, and it is the one the denominator takes on.  The logsumexp uses the
+  // plain unrounded sum.
+  static constexpr bool COMP = COMP_ && TAU > 0.f && !EXPH;
   static constexpr int ELEM = FP8 ? 1 : 2;
   static constexpr int ROW_BYTES = D * ELEM;
   static constexpr int NBOX = ROW_BYTES / 128;
@@ -326,8 +334,9 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
     const int n = pp_kv_tiles<C>(p, qt);
     if (n == 0) continue;
     const int q_idx = qt * C::BM + row;
-    constexpr bool kFusedSum = !C::FP8 && (C::TAU > 0.f || C::EXPH);
+    constexpr bool kFusedSum = !C::FP8 && ((C::TAU > 0.f && !C::COMP) || C::EXPH);
     float m = -INFINITY, l = 0.f, lx = 0.f;   // lx: unrounded row sum (fused path)
+    float lc = 0.f;                           // compensated row sum (COMP)
     float qsc = 1.f, vmax = 1.f;
     // FP8: the V tile scales' max, one load per lane per 32 tiles and a warp reduction;
     // the per-step K and V scales are fetched a step ahead, so their load latency
@@ -388,6 +397,12 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       const float m_new = raise ? m_cand : m;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = raise ? ex2(m - m_use) : 1.f;
+      float l_comp = 0.f;
+      if constexpr (C::COMP) {
+        // the tile's largest probability and its bf16 rounding error
+        const float pt = ex2(m_cand - m_use);
+        l_comp = __bfloat162float(__float2bfloat16_rn(pt)) - pt;
+      }
       const uint64_t c2 = f2_pack(c_j, c_j);
       const uint64_t nm2 = f2_pack(-m_use, -m_use);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
@@ -436,7 +451,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
           f2_unpack(p2, s[c], s[c + 1]);
         }
       };
-      constexpr bool kFused = !C::FP8 && (C::TAU > 0.f || C::EXPH);
+      constexpr bool kFused = kFusedSum;
       if constexpr (kFused) {
         if (need_mask)
           exps_bf16(std::integral_constant<int, 0>{});
@@ -451,6 +466,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
       l = l * alpha + (sa + sb);
+      if constexpr (C::COMP) lc = lc * alpha + (sa + sb) + l_comp;
       if constexpr (kFused) {
         float xa, xb;
         f2_unpack(f2_add(f2_add(accx[0], accx[1]), f2_add(accx[2], accx[3])), xa, xb);
@@ -512,7 +528,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       ++gs;
     }
     if (!ok) break;
-    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / l;
+    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / (C::COMP ? lc : l);
     const bool row_ok = q_idx < p.N;
     if (!(ok = mbar_wait(bar(C::B_ODONE + t), ti & 1, wc, kSiteODone))) break;
     ++ti;
