@@ -64,6 +64,10 @@ def _load() -> ctypes.CDLL:
     L.fa_decode.restype = ctypes.c_int
     L.fa_fwd_kernel_name.argtypes = [i, i]
     L.fa_fwd_kernel_name.restype = ctypes.c_char_p
+    L.fa_fwd_host_workspace_size.argtypes = [i, i, i, i]
+    L.fa_fwd_host_workspace_size.restype = sz
+    L.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
+    L.fa_fwd_host.restype = ctypes.c_int
     L.fa_bwd_fp8_workspace_size.argtypes = [i, i, i, i]
     L.fa_bwd_fp8_workspace_size.restype = sz
     L.fa_bwd_fp8.argtypes = [vp] * 13 + [sz, i, i, i, i, f, i, vp]
@@ -237,6 +241,52 @@ def attention_backward(q, k, v, o, dO, lse, causal: bool = False, scale: float |
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
     fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, scale=scale, causal=causal)
     return dq, dk, dv
+
+
+def fa_fwd_host_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib.fa_fwd_host_workspace_size(B, H, N, d))
+
+
+def fa_fwd_host(q, k, v, o, lse, workspace, scale: float | None = None, causal: bool = False,
+                stream=None):
+    """Forward on host (CPU) bf16 tensors [B, H, N, d]: chunks of heads are copied in,
+    computed and copied out with the copies overlapping the kernels.  o (and lse, fp32
+    [B, H, N], or None) are host tensors written once ``stream`` completes; workspace is a
+    device tensor of fa_fwd_host_workspace_size bytes."""
+    shp = tuple(q.shape)
+    if len(shp) != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shp or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous bf16 tensor of q's shape")
+        if t.is_cuda:
+            raise ValueError(f"{n} must be in host memory")
+    B, H, N, d = shp
+    if lse is not None and (tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32
+                            or lse.is_cuda or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous host fp32 [B, H, N] tensor")
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("workspace must be a device tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                           lse.data_ptr() if lse is not None else None, _ptr(workspace), ws_bytes,
+                           B, H, N, d, sc, 1 if causal else 0, _stream(stream)))
+
+
+def attention_forward_host(q, k, v, causal: bool = False, scale: float | None = None,
+                           device=None):
+    """Allocate page-locked o / lse and the device workspace, run fa_fwd_host on the
+    current stream of ``device`` and wait for it."""
+    B, H, N, d = q.shape
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+    lse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    ws = torch.empty(max(1, fa_fwd_host_workspace_size(B, H, N, d)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fa_fwd_host(q, k, v, o, lse, ws, scale=scale, causal=causal, stream=stream)
+    stream.synchronize()
+    return o, lse
 
 
 def fa_bwd_fp8_workspace_size(B: int, H: int, N: int, d: int) -> int:

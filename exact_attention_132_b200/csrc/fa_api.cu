@@ -59,6 +59,12 @@ struct DeviceInfo {
   unsigned* status = nullptr;
   int* sched = nullptr;                 // g_fa_sched of this device
   std::mutex sched_mu;
+  // host-buffer forward (fa_fwd_host): two copy streams and an event pool, made on first
+  // use; the mutex also keeps concurrent calls from reusing each other's events
+  std::mutex host_mu;
+  bool host_ready = false;
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t host_ev[64] = {};   // >= 1 + 3 * kHostChunks
   cudaStream_t sched_stream[kSchedSlots] = {};
   int sched_used = 0;
 };
@@ -481,6 +487,22 @@ size_t fp8_bwd_tensor_bytes(int B, int H, int N, int d) {
   return (static_cast<size_t>(B) * H * N * d * 2 + 255) & ~static_cast<size_t>(255);
 }
 
+// Host-buffer forward: the heads go through in kHostChunks chunks (fewer for small B*H;
+// more chunks shorten the copy-in before the first kernel and the copy-out after the last),
+// each staged in one of two device slots.  A slot holds Q, K, V, O (bf16) and LSE (fp32)
+// of `hc` heads, each part 256-byte aligned.
+constexpr int kHostChunks = 16;
+static_assert(1 + 3 * kHostChunks <= 64, "host pipeline event pool");
+int host_chunk_heads(int BH) {
+  const int nc = BH < kHostChunks ? BH : kHostChunks;
+  return (BH + nc - 1) / nc;
+}
+size_t host_slot_bytes(int hc, int N, int d) {
+  const size_t t = (static_cast<size_t>(hc) * N * d * 2 + 255) & ~static_cast<size_t>(255);
+  const size_t l = (static_cast<size_t>(hc) * N * 4 + 255) & ~static_cast<size_t>(255);
+  return 4 * t + l;
+}
+
 // ------------------------------------------------------------------ no-allocation backward
 // Fixed scratch for fa_bwd_noalloc: one fp32 D_i per row (B*H*N rows at most
 // FA_BWD_NOALLOC_MAX_ROWS).  It lives in the module image, so every GPU that loads
@@ -721,6 +743,98 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* stream) {
   return fa_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes_, B, H,
                     H > 0 ? H : 1, N, d, scale, causal, stream);
+}
+
+// ------------------------------------------------------------------ host-buffer forward
+size_t fa_fwd_host_workspace_size(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  return 2 * host_slot_bytes(host_chunk_heads(B * H), N, d);
+}
+
+fa_status fa_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                      float* lse_host, void* workspace, size_t workspace_bytes_, int B, int H,
+                      int N, int d, float scale, int causal, void* stream) {
+  bool empty = false;
+  if (fa_status s = check_common(B, H, N, scale, &empty)) return s;
+  if (d != 64 && d != 96 && d != 128 && d != 192 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64, 96, 128, 192, 256)", d);
+  if (empty) return FA_OK;
+  if (!q_host || !k_host || !v_host || !o_host)
+    return fail(FA_ERR_INVALID_ARG, "host tensor pointer is NULL");
+  const void* ptrs[] = {workspace};
+  const char* names[] = {"workspace"};
+  if (fa_status s = check_ptrs(ptrs, names, 1)) return s;
+  const size_t need = fa_fwd_host_workspace_size(B, H, N, d);
+  if (workspace_bytes_ < need)
+    return fail(FA_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes_, need);
+  DeviceInfo* di = nullptr;
+  if (fa_status s = device_info(&di)) return s;
+  std::lock_guard<std::mutex> lock(di->host_mu);
+  if (!di->host_ready) {
+    cudaError_t e = cudaStreamCreateWithFlags(&di->copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&di->copy_out, cudaStreamNonBlocking);
+    for (int i = 0; e == cudaSuccess && i < 64; ++i)
+      e = cudaEventCreateWithFlags(&di->host_ev[i], cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "host pipeline setup");
+    di->host_ready = true;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H, hc = host_chunk_heads(BH), nc = (BH + hc - 1) / hc;
+  const size_t slot = host_slot_bytes(hc, N, d);
+  const size_t tb = (static_cast<size_t>(hc) * N * d * 2 + 255) & ~static_cast<size_t>(255);
+  const size_t head_bytes = static_cast<size_t>(N) * d * 2, head_rows = static_cast<size_t>(N);
+  // events: 0 = entry, then per chunk c: 1 + 3c inputs copied, 2 + 3c forward done,
+  // 3 + 3c outputs copied
+  cudaEvent_t* ev = di->host_ev;
+  auto ck = [&](cudaError_t e, const char* what) -> fa_status {
+    return e == cudaSuccess ? FA_OK : cuda_fail(e, what);
+  };
+  // the copies start after the work already queued on the caller's stream
+  if (fa_status s = ck(cudaEventRecord(ev[0], st), "event record")) return s;
+  if (fa_status s = ck(cudaStreamWaitEvent(di->copy_in, ev[0], 0), "stream wait")) return s;
+  if (fa_status s = ck(cudaStreamWaitEvent(di->copy_out, ev[0], 0), "stream wait")) return s;
+  for (int c = 0; c < nc; ++c) {
+    const int h0 = c * hc, hn = (h0 + hc <= BH) ? hc : BH - h0;
+    uint8_t* base = static_cast<uint8_t*>(workspace) + (c % 2) * slot;
+    void* qd = base;
+    void* kd = base + tb;
+    void* vd = base + 2 * tb;
+    void* od = base + 3 * tb;
+    float* ld = reinterpret_cast<float*>(base + 4 * tb);
+    const size_t off = static_cast<size_t>(h0) * head_bytes, nb = static_cast<size_t>(hn) * head_bytes;
+    // inputs of this slot's previous chunk consumed by its forward
+    if (c >= 2)
+      if (fa_status s = ck(cudaStreamWaitEvent(di->copy_in, ev[2 + 3 * (c - 2)], 0), "stream wait"))
+        return s;
+    const void* src[3] = {q_host, k_host, v_host};
+    void* dst[3] = {qd, kd, vd};
+    for (int t = 0; t < 3; ++t)
+      if (fa_status s = ck(cudaMemcpyAsync(dst[t], static_cast<const uint8_t*>(src[t]) + off, nb,
+                                           cudaMemcpyHostToDevice, di->copy_in), "host-to-device copy"))
+        return s;
+    if (fa_status s = ck(cudaEventRecord(ev[1 + 3 * c], di->copy_in), "event record")) return s;
+    // forward of the chunk, once its inputs are in and the slot's previous outputs are out
+    if (fa_status s = ck(cudaStreamWaitEvent(st, ev[1 + 3 * c], 0), "stream wait")) return s;
+    if (c >= 2)
+      if (fa_status s = ck(cudaStreamWaitEvent(st, ev[3 + 3 * (c - 2)], 0), "stream wait")) return s;
+    if (fa_status s = fa_fwd(qd, kd, vd, od, lse_host ? ld : nullptr, 1, hn, N, d, scale, causal, st))
+      return s;
+    if (fa_status s = ck(cudaEventRecord(ev[2 + 3 * c], st), "event record")) return s;
+    // outputs back to the host
+    if (fa_status s = ck(cudaStreamWaitEvent(di->copy_out, ev[2 + 3 * c], 0), "stream wait")) return s;
+    if (fa_status s = ck(cudaMemcpyAsync(static_cast<uint8_t*>(o_host) + off, od, nb,
+                                         cudaMemcpyDeviceToHost, di->copy_out), "device-to-host copy"))
+      return s;
+    if (lse_host)
+      if (fa_status s = ck(cudaMemcpyAsync(lse_host + static_cast<size_t>(h0) * head_rows, ld,
+                                           static_cast<size_t>(hn) * head_rows * 4,
+                                           cudaMemcpyDeviceToHost, di->copy_out), "device-to-host copy"))
+        return s;
+    if (fa_status s = ck(cudaEventRecord(ev[3 + 3 * c], di->copy_out), "event record")) return s;
+  }
+  // the caller's stream completes only after the last copy out (the copy stream runs
+  // its copies in order)
+  return ck(cudaStreamWaitEvent(st, ev[3 + 3 * (nc - 1)], 0), "stream wait");
 }
 
 // ------------------------------------------------------------------ FP8 backward

@@ -78,6 +78,32 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * fa_fwd_host_workspace_size — device workspace fa_fwd_host needs: two staging slots,
+ * each with Q, K, V, O (bf16) and LSE (fp32) of one chunk of heads.  0 when empty.
+ */
+size_t fa_fwd_host_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_fwd_host — fa_fwd on HOST buffers.  The heads go through in up to 16 chunks: while
+ * one chunk's forward runs on `stream`, the next chunk's Q, K, V are copied in and the
+ * previous chunk's O and LSE copied out, on two copy streams of the library's own, so
+ * the host-to-device copies, the kernels and the device-to-host copies overlap.
+ *   q_host, k_host, v_host   in   bf16 [B,H,N,d] in host memory (page-locked memory
+ *                                 lets the copies overlap; pageable memory works too)
+ *   o_host                   out  bf16 [B,H,N,d] in host memory
+ *   lse_host                 out  fp32 [B,H,N] in host memory, or NULL
+ *   workspace                device scratch of >= fa_fwd_host_workspace_size() bytes,
+ *                            owned by the caller; contents on entry are ignored
+ * Asynchronous like cudaMemcpyAsync: the work is queued in the order of `stream`, and
+ * the results are in o_host / lse_host once `stream` has completed (the stream waits
+ * for the last copy out).  Results equal fa_fwd's.  Errors as fa_fwd, plus
+ * FA_ERR_INVALID_ARG for a NULL host pointer or a small workspace.
+ */
+fa_status fa_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                      float* lse_host, void* workspace, size_t workspace_bytes,
+                      int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
  * fa_fwd_fp8 — FP8 (e4m3, OCP "fn" variant) forward with per-tile scales
  * (mypcrig.com post, section "FA3 の飛躍": per-tile rescaling and block-wise
  * quantisation keep FP8 attention accurate).

@@ -112,6 +112,22 @@ def test_fp8_bwd_argument_errors():
     assert fa.lib.fa_bwd_fp8(*([None] * 13), 0, 1, 2, 0, 128, 0.1, 1, None) == fa.FA_OK
 
 
+def test_host_forward_argument_errors():
+    P = lambda x: ctypes.c_void_p(16 * x)
+    need = fa.fa_fwd_host_workspace_size(2, 8, 1000, 128)
+    assert need > 0 and need % 256 == 0
+    assert fa.fa_fwd_host_workspace_size(0, 8, 1000, 128) == 0
+    st = fa.lib.fa_fwd_host(None, P(1), P(1), P(1), None, P(1), need, 2, 8, 1000, 128, 0.1, 1, None)
+    assert st == fa.FA_ERR_INVALID_ARG and "host" in fa.fa_last_error_string()
+    st = fa.lib.fa_fwd_host(P(1), P(1), P(1), P(1), None, P(1), need - 256, 2, 8, 1000, 128, 0.1, 1,
+                            None)
+    assert st == fa.FA_ERR_INVALID_ARG and "workspace" in fa.fa_last_error_string()
+    st = fa.lib.fa_fwd_host(P(1), P(1), P(1), P(1), None, P(1), need, 2, 8, 1000, 80, 0.1, 1, None)
+    assert st == fa.FA_ERR_UNSUPPORTED
+    assert fa.lib.fa_fwd_host(None, None, None, None, None, None, 0, 2, 8, 0, 128, 0.1, 1,
+                              None) == fa.FA_OK
+
+
 def test_python_wrappers_validate_shapes():
     import torch
     q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
