@@ -573,11 +573,33 @@ fa_status dec_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, DecPlan* pl) {
   pl->bn = d <= 128 ? 128 : 64;
   const int dk = d <= 64 ? 64 : (d <= 128 ? 128 : 256);   // kernel head dim
   pl->n_kt = (Nk + pl->bn - 1) / pl->bn;
-  const long long target = 2ll * di->sms;
-  long long ns = (target + pl->BHkv - 1) / pl->BHkv;
-  if (ns < 1) ns = 1;
-  if (ns > pl->n_kt) ns = pl->n_kt;
-  pl->split_tiles = static_cast<int>((pl->n_kt + ns - 1) / ns);
+  // Splits per head: equal key ranges, CTAs taking items round-robin, so the kernel
+  // lasts (rounds of items) x (longest item).  Pick the split count whose useful share
+  // of that, all key tiles / (rounds x SMs x tiles per item), is within 1 % of the best,
+  // with the fewest items (each item adds a partial result to write and merge).
+  const long long tiles = static_cast<long long>(pl->BHkv) * pl->n_kt;
+  const int max_ns = pl->n_kt < 1024 ? pl->n_kt : 1024;
+  double eff[1025] = {};
+  double best = 0.0;
+  for (int ns = 1; ns <= max_ns; ++ns) {
+    const long long st = (pl->n_kt + ns - 1) / ns;
+    const long long items = static_cast<long long>(pl->BHkv) * ((pl->n_kt + st - 1) / st);
+    const long long rounds = (items + di->sms - 1) / di->sms;
+    eff[ns] = static_cast<double>(tiles) / static_cast<double>(rounds * di->sms * st);
+    if (eff[ns] > best) best = eff[ns];
+  }
+  int pick = 1;
+  long long pick_items = -1;
+  for (int ns = 1; ns <= max_ns; ++ns) {
+    if (eff[ns] < best - 0.01) continue;
+    const long long st = (pl->n_kt + ns - 1) / ns;
+    const long long items = static_cast<long long>(pl->BHkv) * ((pl->n_kt + st - 1) / st);
+    if (pick_items < 0 || items < pick_items) {
+      pick = ns;
+      pick_items = items;
+    }
+  }
+  pl->split_tiles = (pl->n_kt + pick - 1) / pick;
   pl->n_split = (pl->n_kt + pl->split_tiles - 1) / pl->split_tiles;
   const size_t rows = static_cast<size_t>(pl->BHkv) * pl->n_split * pl->R;
   pl->part_o_bytes = (rows * dk * sizeof(float) + 255) & ~static_cast<size_t>(255);
