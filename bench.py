@@ -7,10 +7,14 @@ Headline step: one bf16 causal forward of the workload B=4, H=16, N=4096, d=128
 (scale 1/sqrt(128), 1% of K rows x8), i.e. one fa_fwd launch over inputs already
 resident in HBM (Q, K, V = 201 MB > the 126 MB L2, so no flush is needed between
 steps).  Metric: attention TFLOP/s, counting 4*B*H*N^2*d halved for causal.
+The default 100 steps (about 28 ms) stay ahead of the power cap; the same kernel is
+then run for about a second and reported against the sustained matmul peak
+(roofline.sustained).
 
 Extra lines (same JSON object, key "extras"): forward+backward TFLOP/s for
-B=1 H=8 N=8192 d=64 causal and B=2 H=8 N=16384 d=256, and the FP8 forward for
-B=1 H=32 N=32768 d=128 causal (backward counted as 2.5x forward).
+B=1 H=8 N=8192 d=64 causal and B=2 H=8 N=16384 d=256, the causal forward at N=32768,
+decoding (B=8 Hq=32 Hkv=8 Nk=32768) against the HBM peak, and the FP8 forward and
+backward for B=1 H=32 N=32768 d=128 causal (backward counted as 2.5x forward).
 
 With N GPUs (torchrun, one process per GPU) every rank runs its own copy of the
 workload (independent heads: no data-path collective); value = all ranks' FLOPs
@@ -193,6 +197,17 @@ def run_ours(args):
     achieved = flops / (kernel_ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # The same kernel back to back for about a second: after some 60 ms at full load the
+    # 1 kW power cap lowers the clock, so this is compared with the sustained matmul peak
+    # (the burst figure above fits the short timed region)
+    sus_steps = max(1, int(1000.0 / max(kernel_ms, 1e-3)))
+    sclocks = ClockSampler(local)
+    sclocks.start()
+    sus_ms, sus_per = time_steps(step, sus_steps, 0, stream)
+    sclk = sclocks.stop()
+    sus_kernel_ms = statistics.mean(sus_per)
+    sus_achieved = flops / (sus_kernel_ms * 1e-3) / 1e12
+    sus_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
 
     # end to end through the public API with host buffers (fa_fwd_host): every step
     # copies Q, K, V in from page-locked memory and O, LSE out, chunk by chunk, the
@@ -246,7 +261,11 @@ def run_ours(args):
                      "kernel": kname,
                      "kernel_ms": round(kernel_ms, 4),
                      "traffic": FWD_TRAFFIC_BYTES.get(kernel_source_hash(kname)),
-                     "kernel_source_hash": kernel_source_hash(kname)},
+                     "kernel_source_hash": kernel_source_hash(kname),
+                     "sustained": {"steps": sus_steps, "achieved": round(sus_achieved, 2),
+                                   "peak": sus_peak, "frac": round(sus_achieved / sus_peak, 4),
+                                   "peak_source": f"{peak_src} bf16 dense matmul (sustained)",
+                                   "clocks": sclk}},
         "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "ms_per_step": round(e2e_ms / e2e_steps, 4)},
@@ -476,7 +495,7 @@ def main():
                     help="only launch this workload's kernels (--profile-launches times) for ncu")
     ap.add_argument("--profile-launches", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
