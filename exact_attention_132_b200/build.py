@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfa.so")
 SOURCES = ["fa_api.cu"]
-HEADERS = ["sm100_ptx.cuh", "fa_fwd.cuh", "fa_fwd_pp.cuh", "fa_fwd_ws.cuh", "fa_fwd_sp.cuh", "fa_decode.cuh", "fa_bwd.cuh"]
+HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))   # every kernel header
 
 
 def nvcc_path() -> str:

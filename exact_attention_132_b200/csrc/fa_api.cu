@@ -17,7 +17,6 @@
 #include "fa_fwd.cuh"
 #include "fa_fwd_pp.cuh"
 #include "fa_fwd_ws.cuh"
-#include "fa_fwd_sp.cuh"
 #include "fa_decode.cuh"
 #include "fa_dequant.cuh"
 #include "sm100_ptx.cuh"
@@ -256,12 +255,7 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
   if (fa_status s = make_map(&mq, q, C::FP8, p.ld, p.N, p.BH, C::BM)) return s;
   if (fa_status s = make_map(&mk, k, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
   if (fa_status s = make_map(&mv, v, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
-  auto kern = [] {
-    if constexpr (C::SEPARATE_P)
-      return fa_fwd_sp_kernel<C>;
-    else
-      return fa_fwd_ws_kernel<C>;
-  }();
+  auto kern = fa_fwd_ws_kernel<C>;
   if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
   p.n_qt = (p.N + C::BM - 1) / C::BM;
   p.n_kt = (p.N + C::BN - 1) / C::BN;
@@ -301,9 +295,6 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #ifndef FA_FWD_WS_SPLIT
 #define FA_FWD_WS_SPLIT 0
 #endif
-#ifndef FA_FWD_SP_SPLIT
-#define FA_FWD_SP_SPLIT 1
-#endif
 #ifndef FA_FWD_D128_KST
 #define FA_FWD_D128_KST 2
 #endif
@@ -327,7 +318,7 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #endif
 // Kernel family per problem class (measured fastest on the causal N = 4096 workloads):
 // 0 = one query tile per CTA (fa_fwd.cuh), 1 = two query tiles (fa_fwd_pp.cuh),
-// 2 = split softmax (fa_fwd_ws.cuh), 3 = separate P buffers (fa_fwd_sp.cuh).
+// 2 = split softmax (fa_fwd_ws.cuh).
 #ifndef FA_FWD_D64_KIND
 #define FA_FWD_D64_KIND 1
 #endif
@@ -348,14 +339,13 @@ struct FwdPick {
       KIND == 0, FwdCfg<D, 128, kWide ? 3 : 4, kWide ? 2 : 4, FP8, EMU>,
       std::conditional_t<
           KIND == 1, PPCfg<D, KST, VST, FP8, EMU, FA_FWD_TAU, FA_FWD_EXPH, FA_FWD_PP_COMP != 0>,
-          std::conditional_t<KIND == 2,
-                             WSCfg<D, KST, VST, FP8, EMU, EMU,
-                                   FA_FWD_WS_SPLIT != 0, FA_FWD_WS_INDEP != 0, FA_FWD_WS_TAU>,
-                             SPCfg<D, KST, VST, FP8, EMU, FA_FWD_SP_SPLIT != 0>>>>;
+          WSCfg<D, KST, VST, FP8, EMU, EMU, FA_FWD_WS_SPLIT != 0, FA_FWD_WS_INDEP != 0,
+                FA_FWD_WS_TAU>>>;
+  static_assert(KIND >= 0 && KIND <= 2, "kernel family 0, 1 or 2");
   static const char* name() {
     static const std::string n = [] {
       static const char* fam[] = {"fa_fwd_kernel<FwdCfg", "fa_fwd_pp_kernel<PPCfg",
-                                  "fa_fwd_ws_kernel<WSCfg", "fa_fwd_sp_kernel<SPCfg"};
+                                  "fa_fwd_ws_kernel<WSCfg"};
       char buf[128];
       std::snprintf(buf, sizeof buf, "%s<%d,KST%d,VST%d,%s>>", fam[KIND], D, Cfg::KST, Cfg::VST,
                     FP8 ? "e4m3" : "bf16");

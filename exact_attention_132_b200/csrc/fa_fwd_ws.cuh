@@ -45,7 +45,6 @@ struct WSCfg {
   // own output accumulator O_h (h = column half of the scores), so the two halves of a
   // row never wait for each other inside the key loop; they are combined once per tile.
   static constexpr bool INDEP = INDEP_;
-  static constexpr bool SEPARATE_P = false;
   // bf16, independent halves only: a row's reference max moves (and O_h is rescaled)
   // only when the row max exceeds it by more than TAU (log2 units), so P <= 2^TAU.  O is
   // then normalised by the sum of the bf16-ROUNDED probabilities, the very values the
