@@ -1,0 +1,54 @@
+"""Dynamic work distribution of the forward kernels: per-stream item counters that every
+launch leaves at zero.  Back-to-back launches on one stream and overlapping launches on
+several streams must each compute every item exactly once (results equal a lone launch)."""
+import pytest
+import torch
+
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fa():
+    import exact_attention_132_b200 as m
+    return m
+
+
+def _inputs(B, H, N, d, causal, seed):
+    w = workloads.make_small(B, H, N, d, causal, seed=seed, backward=False)
+    return w, [t.cuda() for t in workloads.make_bf16_inputs(w, with_grad_out=False)]
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_back_to_back_launches_on_one_stream(fa, d):
+    w, (q, k, v) = _inputs(2, 4, 1000, d, True, seed=d)
+    ref_o, ref_l = fa.attention_forward(q, k, v, causal=True, scale=w.sm_scale)
+    o, lse = torch.empty_like(ref_o), torch.empty_like(ref_l)
+    for _ in range(20):
+        o.zero_()
+        fa.fa_fwd(q, k, v, o, lse, scale=w.sm_scale, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref_o) and torch.equal(lse, ref_l)
+    assert fa.fa_get_device_status() == 0
+
+
+def test_overlapping_launches_on_several_streams(fa):
+    # causal d=128 (two-tile kernel) and d=256 (one-tile kernel) problems, each on its
+    # own stream, launched repeatedly so that their kernels overlap on the GPU
+    probs = [_inputs(4, 8, 2048, 128, True, seed=1), _inputs(1, 8, 2048, 256, True, seed=2),
+             _inputs(2, 8, 1536, 64, False, seed=3)]
+    refs = [fa.attention_forward(q, k, v, causal=w.causal, scale=w.sm_scale)
+            for w, (q, k, v) in probs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in probs]
+    outs = [(torch.empty_like(r[0]), torch.empty_like(r[1])) for r in refs]
+    for _ in range(10):
+        for (w, (q, k, v)), (o, lse), s in zip(probs, outs, streams):
+            with torch.cuda.stream(s):
+                o.zero_()
+                fa.fa_fwd(q, k, v, o, lse, scale=w.sm_scale, causal=w.causal, stream=s)
+    torch.cuda.synchronize()
+    for (o, lse), (ro, rl) in zip(outs, refs):
+        assert torch.equal(o, ro) and torch.equal(lse, rl)
+    assert fa.fa_get_device_status() == 0
