@@ -274,17 +274,17 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 
 // Tuning knobs (compile-time): software-exp2 share, pipeline depth, kernel family.
 // software-exp2 share (quarters of the exponentials) per problem class, measured: the
-// two-tile kernel gains from 2 at d = 64 and FP8 but wants none at bf16 d = 128 (its
-// per-step path is issue-bound there, not bound by the special-function unit); the
-// d = 256 kernel (tensor-core bound) none
+// two-tile kernel wants 1 at d = 64 and FP8 (2 and 3 were slower) and none at bf16
+// d = 128 (its per-step path is issue-bound there, not bound by the special-function
+// unit); the d = 256 kernel (tensor-core bound) none
 #ifndef FA_FWD_EMU
 #define FA_FWD_EMU 0
 #endif
 #ifndef FA_FWD_D64_EMU
-#define FA_FWD_D64_EMU 2
+#define FA_FWD_D64_EMU 1
 #endif
 #ifndef FA_FWD_F8_EMU
-#define FA_FWD_F8_EMU 2
+#define FA_FWD_F8_EMU 1
 #endif
 #ifndef FA_FWD_D256_EMU
 #define FA_FWD_D256_EMU 0
@@ -369,18 +369,22 @@ using FwdF8D128 = FwdPick<FA_FWD_F8_KIND, 128, true, FA_FWD_F8_EMU>;
 using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_D256_EMU>;
 using FwdF8D256 = FwdCfg<256, 128, 3, 2, true, FA_FWD_F8_EMU>;
 
+// backward software-exp2 share: a quarter at d = 64 and 128, none at d = 256 (measured)
 #ifndef FA_BWD_EMU
 #define FA_BWD_EMU 1
+#endif
+#ifndef FA_BWD_D256_EMU
+#define FA_BWD_D256_EMU 0
 #endif
 #ifndef FA_BWD_D64_STAGES
 #define FA_BWD_D64_STAGES 3
 #endif
 using DkdvD64 = DkdvCfg<64, 64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU>;
 using DkdvD128 = DkdvCfg<128, 128, 64, 3, 3, 2, 2, FA_BWD_EMU>;
-using DkdvD256 = DkdvCfg<256, 128, 64, 2, 1, 2, 2, FA_BWD_EMU>;
+using DkdvD256 = DkdvCfg<256, 128, 64, 2, 1, 2, 2, FA_BWD_D256_EMU>;
 using DqD64 = DqCfg<64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU>;
 using DqD128 = DqCfg<128, 128, 2, 2, 2, 1, FA_BWD_EMU>;
-using DqD256 = DqCfg<256, 64, 2, 1, 2, 2, FA_BWD_EMU>;
+using DqD256 = DqCfg<256, 64, 2, 1, 2, 2, FA_BWD_D256_EMU>;
 
 template <class CK, class CQ>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
