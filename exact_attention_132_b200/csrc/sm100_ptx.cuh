@@ -132,7 +132,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 // 3-D tiled bulk tensor load global -> shared, completion counted in bytes on `bar`.
-// No cluster multicast.
+// The destination is this CTA's own shared memory only.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
                                             int x, int y, int z) {
   asm volatile(
