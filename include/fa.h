@@ -71,6 +71,11 @@ typedef enum {
  *                                  (the normalisation statistic the backward reuses;
  *                                  issoh.co.jp page, section 逆伝播でL×L行列を保存せず
  *                                  再計算する設計).  May be NULL if not wanted.
+ * Work distribution: the CTAs draw work items from a counter the library keeps per
+ * stream (and per device); each launch leaves it at zero when it ends.  Launches in one
+ * stream run one after the other and share it, launches in different streams have
+ * their own.  A CUDA graph captured from this call keeps the counter of the capturing
+ * stream, so two replays of it must not run at the same time.
  * Returns FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED (d not 64/96/128/192/256) or
  * FA_ERR_CUDA.
  */
