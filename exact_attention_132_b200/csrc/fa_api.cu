@@ -619,8 +619,8 @@ fa_status launch_decode(const void* q, const void* k, const void* v, void* o, fl
   kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode split kernel launch");
-  const long long warps = static_cast<long long>(p.BHkv) * p.R;
-  const long long blocks = (warps * 32 + 255) / 256;
+  const long long threads = static_cast<long long>(p.BHkv) * p.R * (C::D / 4);
+  const long long blocks = (threads + 255) / 256;
   fa_decode_combine_kernel<C::D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, o, lse);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode combine kernel launch");

@@ -387,43 +387,54 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 }
 
 // ---------------------------------------------------------------- combine
-// One warp per query row of a group: lse = log sum_s exp(lse_s) and
-// O = sum_s exp(lse_s - lse) O_s, written as bf16 (and lse as fp32).  Memory-bound
-// and small next to the split kernel (n_split rows of d fp32 per output row).
+// lse = log sum_s exp(lse_s) and O = sum_s exp(lse_s - lse) O_s per query row, written as
+// bf16 (and lse as fp32).  One thread per (row, four output columns): every thread reads
+// its row's split logsumexps (cached after the first thread) and then the partial values
+// of its columns from all splits, several loads in flight, so the merge costs a few
+// memory round trips rather than one per split.
 template <int D>
 __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecParams p, void* o, float* lse) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
-  const int lane = threadIdx.x & 31;
-  if (warp >= p.BHkv * p.R) return;
-  const int bh = warp / p.R, row = warp - bh * p.R;
+  constexpr int C4 = D / 4;                       // float4 groups per row
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<long long>(p.BHkv) * p.R * C4) return;
+  const int c4 = static_cast<int>(t % C4);
+  const long long rr = t / C4;
+  const int row = static_cast<int>(rr % p.R);
+  const int bh = static_cast<int>(rr / p.R);
   const float* pl = p.part_lse + static_cast<size_t>(bh) * p.n_split * p.R + row;
   float mx = -INFINITY;
-  for (int s = lane; s < p.n_split; s += 32) mx = fmaxf(mx, pl[static_cast<size_t>(s) * p.R]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+#pragma unroll 8
+  for (int s = 0; s < p.n_split; ++s) mx = fmaxf(mx, __ldg(pl + static_cast<size_t>(s) * p.R));
   // every row sees at least one key, so mx is finite
   float sum = 0.f;
-  for (int s = lane; s < p.n_split; s += 32) sum += __expf(pl[static_cast<size_t>(s) * p.R] - mx);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+#pragma unroll 8
+  for (int s = 0; s < p.n_split; ++s) sum += __expf(__ldg(pl + static_cast<size_t>(s) * p.R) - mx);
   const float lse_row = mx + __logf(sum);
-  constexpr int PER = D / 32;                     // output columns per lane
-  float acc[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  const float4* src = reinterpret_cast<const float4*>(
+      p.part_o + (static_cast<size_t>(bh) * p.n_split * p.R + row) * D) + c4;
+  const size_t split_stride = static_cast<size_t>(p.R) * C4;   // float4s between splits
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
   for (int s = 0; s < p.n_split; ++s) {
-    const float ls = pl[static_cast<size_t>(s) * p.R];
-    if (ls == -INFINITY) continue;
-    const float wgt = __expf(ls - lse_row);
-    const float* src = p.part_o + ((static_cast<size_t>(bh) * p.n_split + s) * p.R + row) * D;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = fmaf(wgt, src[lane + 32 * i], acc[i]);
+    const float ls = __ldg(pl + static_cast<size_t>(s) * p.R);
+    const float w = ls == -INFINITY ? 0.f : __expf(ls - lse_row);   // a split with no key
+    const float4 v = __ldg(src + s * split_stride);
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z);
+    acc.w = fmaf(w, v.w, acc.w);
   }
-  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o) + (static_cast<size_t>(bh) * p.R + row) * p.ld;
-#pragma unroll
-  for (int i = 0; i < PER; ++i)
-    if (lane + 32 * i < p.ld) dst[lane + 32 * i] = __float2bfloat16_rn(acc[i]);
-  if (lse != nullptr && lane == 0) lse[static_cast<size_t>(bh) * p.R + row] = lse_row;
+  const int col = 4 * c4;
+  if (col < p.ld) {
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o) + (static_cast<size_t>(bh) * p.R + row) * p.ld + col;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(dst) = pk;   // ld is a multiple of 16, so 8-byte aligned
+  }
+  if (lse != nullptr && c4 == 0) lse[static_cast<size_t>(bh) * p.R + row] = lse_row;
 }
 
 }  // namespace fa
