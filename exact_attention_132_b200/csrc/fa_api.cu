@@ -289,6 +289,10 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #ifndef FA_FWD_D256_EMU
 #define FA_FWD_D256_EMU 0
 #endif
+// d = 256 (one-tile kernel): rescale threshold with the compensated row sum
+#ifndef FA_FWD_D256_TAU
+#define FA_FWD_D256_TAU 8
+#endif
 #ifndef FA_FWD_WS_INDEP
 #define FA_FWD_WS_INDEP 1
 #endif
@@ -366,7 +370,7 @@ struct FwdPick {
 using FwdD64 = FwdPick<FA_FWD_D64_KIND, 64, false, FA_FWD_D64_EMU>;
 using FwdD128 = FwdPick<FA_FWD_D128_KIND, 128, false, FA_FWD_EMU>;
 using FwdF8D128 = FwdPick<FA_FWD_F8_KIND, 128, true, FA_FWD_F8_EMU>;
-using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_D256_EMU>;
+using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_D256_EMU, FA_FWD_D256_TAU>;
 using FwdF8D256 = FwdCfg<256, 128, 3, 2, true, FA_FWD_F8_EMU>;
 
 // backward software-exp2 share: a quarter at d = 64 and 128, none at d = 256 (measured)

@@ -73,7 +73,7 @@ __device__ __forceinline__ int fwd_kv_head(const FwdParams& p, int bh) {
   return b * (p.H / p.g) + (bh - b * p.H) / p.g;
 }
 
-template <int D_, int BN_, int KST_, int VST_, bool FP8_, int EMU_ = 1>
+template <int D_, int BN_, int KST_, int VST_, bool FP8_, int EMU_ = 1, int TAU_ = 0>
 struct FwdCfg {
   static constexpr int D = D_;
   static constexpr int BN = BN_;
@@ -85,11 +85,13 @@ struct FwdCfg {
   // Of every 4 column pairs of a score row, EMU take their exponentials on the FMA
   // pipe (ex2_poly_pair), the rest on the special-function unit.
   static constexpr int EMU = EMU_;
-  // Reference-max slack in log2 units: the running max used for the exponentials
-  // moves (and O is rescaled) only when a row max exceeds it by more than TAU.  0 =
-  // rescale exactly when the max changes: with TAU > 0 the largest probability of a
-  // row is no longer exactly 1.0 and its bf16 rounding shows in O.
-  static constexpr float TAU = 0.f;
+  // Reference-max slack in log2 units (bf16 only): the running max used for the
+  // exponentials moves (and O is rescaled) only when a row max exceeds it by more than
+  // TAU.  With TAU > 0 the largest probability of a row is no longer exactly 1.0, so
+  // the row sum that normalises O takes on, per key tile, the bf16 rounding error of
+  // the tile's largest probability, as the P V product does (the logsumexp keeps the
+  // plain unrounded sum).
+  static constexpr float TAU = FP8_ ? 0.f : static_cast<float>(TAU_);
   static constexpr int BM = 128;
   static constexpr int ELEM = FP8 ? 1 : 2;
   static constexpr int ROW_BYTES = D * ELEM;        // bytes of one tile row
@@ -407,6 +409,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
     const int n = fwd_num_kv_tiles<C>(p, qt);
     const int q_idx = qt * C::BM + row;
     float m = -INFINITY, l = 0.f;
+    float lc = 0.f;                               // compensated row sum (TAU > 0)
     float qsc = 1.f, vmax = 1.f;
     if constexpr (C::FP8) {
       static_assert(!C::FP8 || C::BN == 128, "FP8 key tile = one 128-row scale tile");
@@ -466,6 +469,12 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
       const float m_new = raise ? m_cand : m;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = raise ? ex2(m - m_use) : 1.f;   // 0 on the first tile (m = -inf)
+      float l_comp = 0.f;
+      if constexpr (C::TAU > 0.f) {
+        // the tile's largest probability and its bf16 rounding error
+        const float pt = ex2(m_cand - m_use);
+        l_comp = __bfloat162float(__float2bfloat16_rn(pt)) - pt;
+      }
       // P = 2^(S c - m): pairs through the f32x2 FMA; most exponentials on the
       // special-function unit, EMU of every 4 pairs on the FMA pipe.
       const uint64_t c2 = f2_pack(c_j, c_j);
@@ -497,6 +506,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
       l = l * alpha + (sa + sb);
+      if constexpr (C::TAU > 0.f) lc = lc * alpha + (sa + sb) + l_comp;
       // P -> tensor memory over the consumed S columns
       if constexpr (C::FP8) {
 #pragma unroll
@@ -544,7 +554,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, co
     const uint32_t glast = g + n - 1;
     if (!(ok = mbar_wait(bar(C::B_ODONE), glast & 1, wc, kSiteODone))) break;
     tc_fence_after();
-    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / l;
+    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / (C::TAU > 0.f ? lc : l);
     const bool row_ok = q_idx < p.N;
     __nv_bfloat16* orow = o_out + (static_cast<size_t>(bh) * p.N + q_idx) * p.ld;
 #pragma unroll 1
