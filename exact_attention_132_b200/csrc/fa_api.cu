@@ -625,8 +625,19 @@ fa_status launch_decode(const void* q, const void* k, const void* v, void* o, fl
   if (e != cudaSuccess) return cuda_fail(e, "decode split kernel launch");
   const long long threads = static_cast<long long>(p.BHkv) * p.R * (C::D / 4);
   const long long blocks = (threads + 255) / 256;
-  fa_decode_combine_kernel<C::D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, o, lse);
-  e = cudaGetLastError();
+  // programmatic dependent launch: the merge kernel is scheduled while the split kernel
+  // finishes and waits for it on the device (griddepcontrol.wait), which hides its launch
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, fa_decode_combine_kernel<C::D>, p, o, lse);
   if (e != cudaSuccess) return cuda_fail(e, "decode combine kernel launch");
   return FA_OK;
 }

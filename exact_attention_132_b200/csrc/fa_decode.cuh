@@ -392,8 +392,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // its row's split logsumexps (cached after the first thread) and then the partial values
 // of its columns from all splits, several loads in flight, so the merge costs a few
 // memory round trips rather than one per split.
+// Launched as a programmatic dependent of the split kernel: its blocks start while the
+// split kernel's last CTAs run, and wait here until that grid has completed and its
+// partial results are visible.
 template <int D>
 __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecParams p, void* o, float* lse) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int C4 = D / 4;                       // float4 groups per row
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= static_cast<long long>(p.BHkv) * p.R * C4) return;
