@@ -52,3 +52,37 @@ def test_overlapping_launches_on_several_streams(fa):
     for (o, lse), (ro, rl) in zip(outs, refs):
         assert torch.equal(o, ro) and torch.equal(lse, rl)
     assert fa.fa_get_device_status() == 0
+
+
+def test_forward_and_decode_replay_from_a_cuda_graph(fa):
+    """Captured once and replayed: each replay must draw its work items afresh (the
+    counter is back at zero after every launch) and the decode merge must still wait for
+    its split kernel."""
+    w, (q, k, v) = _inputs(2, 8, 1500, 128, True, seed=31)
+    o_ref, l_ref = fa.attention_forward(q, k, v, causal=True, scale=w.sm_scale)
+    kd, vd = k[:, :2].contiguous(), v[:, :2].contiguous()
+    qd = q[:, :, -2:].contiguous()
+    od_ref, ld_ref = fa.attention_decode(qd, kd, vd, causal=True, scale=w.sm_scale)
+    torch.cuda.synchronize()
+    o, lse = torch.empty_like(o_ref), torch.empty_like(l_ref)
+    od, ld = torch.empty_like(od_ref), torch.empty_like(ld_ref)
+    ws = torch.empty(fa.fa_decode_workspace_size(2, 8, 2, 2, 1500, 128), dtype=torch.uint8,
+                     device="cuda")
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        # warm-up outside the capture (first-use setup such as kernel attributes)
+        fa.fa_fwd(q, k, v, o, lse, scale=w.sm_scale, causal=True, stream=s)
+        fa.fa_decode(qd, kd, vd, od, ld, ws, scale=w.sm_scale, causal=True, stream=s)
+    s.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        fa.fa_fwd(q, k, v, o, lse, scale=w.sm_scale, causal=True, stream=s)
+        fa.fa_decode(qd, kd, vd, od, ld, ws, scale=w.sm_scale, causal=True, stream=s)
+    for _ in range(5):
+        o.zero_()
+        od.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
+        assert torch.equal(od, od_ref) and torch.equal(ld, ld_ref)
+    assert fa.fa_get_device_status() == 0
