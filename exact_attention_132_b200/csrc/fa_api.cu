@@ -390,6 +390,25 @@ using DqD64 = DqCfg<64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_
 using DqD128 = DqCfg<128, 128, 2, 2, 2, 1, FA_BWD_EMU>;
 using DqD256 = DqCfg<256, 64, 2, 1, 2, 2, FA_BWD_D256_EMU>;
 
+// Launch `kern` as a programmatic dependent of the previous kernel in `stream`: it may
+// be scheduled before that kernel ends; the kernel itself waits (griddepcontrol.wait)
+// where it needs the previous one's results.
+template <class K, class... Args>
+cudaError_t launch_dependent(K kern, unsigned grid, unsigned threads, int smem, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <class CK, class CQ>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                      BwdParams p, cudaStream_t stream) {
@@ -435,8 +454,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     pk.group_heads = causal_group_heads(p.BH / p.g, 4ll * p.g * p.N * p.ld);
     // one CTA per key/value head, key tile and d part
     const long long grid = static_cast<long long>(p.BH / p.g) * pk.n_kt * CK::NSPLIT;
-    kern<<<static_cast<unsigned>(grid), CK::THREADS, CK::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, pk);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_dependent(kern, static_cast<unsigned>(grid), CK::THREADS, CK::SMEM_ALLOC,
+                                     stream, mq, mk, mv, mdo, pk);
     if (e != cudaSuccess) return cuda_fail(e, "dK/dV kernel launch");
   }
   // 3. dQ
@@ -453,7 +472,9 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     pq.n_kt = (p.N + CQ::BN - 1) / CQ::BN;
     pq.group_heads = causal_group_heads(p.BH, 4ll * p.N * p.ld);   // K and V of the head
     const long long grid = static_cast<long long>(p.BH) * pq.n_qt;
-    kern<<<static_cast<unsigned>(grid), CQ::THREADS, CQ::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, pq);
+    cudaError_t e0 = launch_dependent(kern, static_cast<unsigned>(grid), CQ::THREADS,
+                                      CQ::SMEM_ALLOC, stream, mq, mk, mv, mdo, pq);
+    if (e0 != cudaSuccess) return cuda_fail(e0, "dQ kernel launch");
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "dQ kernel launch");
   }

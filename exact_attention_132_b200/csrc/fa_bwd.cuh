@@ -215,11 +215,16 @@ __device__ __forceinline__ void exp2_row(const uint32_t (&r)[N], float c, float 
   }
 }
 
+// Launched as a programmatic dependent of the row-dot pass: it waits for that grid (its
+// D_i rows) before anything else, then lets the dQ pass be scheduled, so the dQ CTAs
+// fill the SMs this pass's last wave leaves idle (the two passes are independent).
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     fa_bwd_dkdv(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                 const BwdParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -851,6 +856,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
   }
+  // This pass may start before the dK/dV pass ends (it reads nothing that pass writes);
+  // it ends only after it, so work queued behind the backward sees dK and dV complete.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace fa
