@@ -425,3 +425,31 @@ def attention_backward_gqa(q, k, v, o, dO, lse, causal: bool = False, scale: flo
     ws = torch.empty(max(fa_bwd_workspace_size(B, Hq, N, d), 16), dtype=torch.uint8, device=q.device)
     fa_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, ws, scale=scale, causal=causal)
     return dq, dk, dv
+
+
+# ------------------------------------------------------------------ autograd
+class _Attention(torch.autograd.Function):
+    """O = softmax(scale Q K^T) V with the library's forward, and its backward by
+    recomputation from the saved logsumexp.  Grouped heads when K and V have fewer
+    heads than Q."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, causal, scale):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, lse = attention_forward_gqa(q, k, v, causal=causal, scale=scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.causal, ctx.scale = causal, scale
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = attention_backward_gqa(q, k, v, o, do.contiguous(), lse, causal=ctx.causal,
+                                            scale=ctx.scale)
+        return dq, dk, dv, None, None
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None):
+    """Differentiable exact attention on bf16 CUDA tensors q [B, Hq, N, d], k and v
+    [B, Hkv, N, d] (Hq a multiple of Hkv); scale defaults to 1/sqrt(d)."""
+    return _Attention.apply(q, k, v, causal, scale)
