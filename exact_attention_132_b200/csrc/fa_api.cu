@@ -139,6 +139,23 @@ fa_status make_map(CUtensorMap* m, const void* ptr, bool fp8, int d, int N, int 
   return FA_OK;
 }
 
+// fp32 [BH, N, d] tensor (the fused backward's dQ sums) in 32 x 32 boxes, 128-byte
+// swizzle: the target of the compute warps' reduce-adds.
+fa_status make_map_f32(CUtensorMap* m, void* ptr, int d, int N, int BH) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(N) * d * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FA_OK;
+}
+
 // Set the dynamic shared-memory limit of a kernel once per device.  `Tag` makes the
 // cache per kernel: every kernel here has the same signature, so K alone does not.
 template <class Tag, class K>
@@ -383,7 +400,14 @@ using FwdF8D256 = FwdCfg<256, 128, 3, 2, true, FA_FWD_F8_EMU>;
 #ifndef FA_BWD_D64_STAGES
 #define FA_BWD_D64_STAGES 3
 #endif
+// d = 64: dQ accumulated by the dK/dV pass (fp32 atomics into the workspace) instead of
+// a dQ pass of its own
+#ifndef FA_BWD_D64_FUSED
+#define FA_BWD_D64_FUSED 1
+#endif
 using DkdvD64 = DkdvCfg<64, 64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU>;
+using DkdvD64F =
+    DkdvCfg<64, 64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU, true>;
 using DkdvD128 = DkdvCfg<128, 128, 64, 3, 3, 2, 2, FA_BWD_EMU>;
 using DkdvD256 = DkdvCfg<256, 128, 64, 2, 1, 2, 2, FA_BWD_D256_EMU>;
 using DqD64 = DqCfg<64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU>;
@@ -426,7 +450,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       if (blocks > cap) blocks = cap;
       kern<<<static_cast<int>(blocks), 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO),
-          const_cast<float*>(p.drow), rows);
+          const_cast<float*>(p.drow), rows, CK::FUSEDQ ? p.dq_acc : nullptr);
     };
     static_assert(D == 64 || D == 128 || D == 256, "kernel head dims");
     if (p.ld == D)
@@ -445,6 +469,10 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     if (fa_status s = make_map(&mdo, dO, false, p.ld, p.N, p.BH, CK::BMQ)) return s;
     if (fa_status s = make_map(&mk, k, false, p.ld, p.N, p.BH / p.g, CK::BN)) return s;
     if (fa_status s = make_map(&mv, v, false, p.ld, p.N, p.BH / p.g, CK::BN)) return s;
+    CUtensorMap mdq = mq;                 // the dQ sums' map (fused path; unused otherwise)
+    if constexpr (CK::FUSEDQ) {
+      if (fa_status s = make_map_f32(&mdq, p.dq_acc, D, p.N, p.BH)) return s;
+    }
     auto kern = fa_bwd_dkdv<CK>;
     if (fa_status s = prepare_kernel<CK>(kern, CK::SMEM_ALLOC)) return s;
     BwdParams pk = p;
@@ -455,8 +483,20 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     // one CTA per key/value head, key tile and d part
     const long long grid = static_cast<long long>(p.BH / p.g) * pk.n_kt * CK::NSPLIT;
     cudaError_t e = launch_dependent(kern, static_cast<unsigned>(grid), CK::THREADS, CK::SMEM_ALLOC,
-                                     stream, mq, mk, mv, mdo, pk);
+                                     stream, mq, mk, mv, mdo, mdq, pk);
     if (e != cudaSuccess) return cuda_fail(e, "dK/dV kernel launch");
+  }
+  if constexpr (CK::FUSEDQ) {
+    // 4. dQ = scale dQ_acc (the dK/dV pass summed it)
+    const long long n8 = static_cast<long long>(p.BH) * p.N * D / 8;
+    long long blocks = (n8 + 255) / 256;
+    const long long cap = static_cast<long long>(di->sms) * 8;
+    if (blocks > cap) blocks = cap;
+    cudaError_t e = launch_dependent(fa_bwd_dq_convert, static_cast<unsigned>(blocks), 256, 0, stream,
+                                     static_cast<const float*>(p.dq_acc),
+                                     static_cast<__nv_bfloat16*>(p.dq), n8, p.scale);
+    if (e != cudaSuccess) return cuda_fail(e, "dQ convert kernel launch");
+    return FA_OK;
   }
   // 3. dQ
   {
@@ -499,6 +539,15 @@ __global__ void wait_selftest_kernel(unsigned* status, unsigned long long timeou
 size_t workspace_bytes(int B, int H, int N) {
   const size_t rows = static_cast<size_t>(B) * H * N;
   return (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+// The backward's workspace: D_i rows, then (fused d = 64 path) the fp32 dQ sums.
+bool bwd_fused_dq(int d) { return FA_BWD_D64_FUSED != 0 && d == 64; }
+size_t bwd_workspace_need(int B, int H, int N, int d) {
+  size_t n = workspace_bytes(B, H, N);
+  if (bwd_fused_dq(d))
+    n += (static_cast<size_t>(B) * H * N * d * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  return n;
 }
 
 // FP8 backward: one bf16 [B,H,N,d] copy of a dequantised input, 256-byte aligned
@@ -745,9 +794,8 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  (void)d;
   if (B <= 0 || H <= 0 || N <= 0) return 0;
-  return workspace_bytes(B, H, N);
+  return bwd_workspace_need(B, H, N, d);
 }
 
 fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
@@ -764,9 +812,9 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
   const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv, workspace};
   const char* names[] = {"q", "k", "v", "o", "dO", "lse", "dq", "dk", "dv", "workspace"};
   if (fa_status s = check_ptrs(ptrs, names, 10)) return s;
-  if (workspace_bytes_ < workspace_bytes(B, Hq, N))
+  if (workspace_bytes_ < bwd_workspace_need(B, Hq, N, d))
     return fail(FA_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes_,
-                workspace_bytes(B, Hq, N));
+                bwd_workspace_need(B, Hq, N, d));
   BwdParams p{};
   p.BH = B * Hq;
   p.H = Hq;
@@ -777,12 +825,17 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
   p.scale = scale;
   p.lse = lse;
   p.drow = static_cast<const float*>(workspace);
+  p.dq_acc = bwd_fused_dq(d) ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                        workspace_bytes(B, Hq, N))
+                             : nullptr;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 64: return launch_bwd<DkdvD64, DqD64>(q, k, v, o, dO, p, st);
+    case 64:
+      if (bwd_fused_dq(d)) return launch_bwd<DkdvD64F, DqD64>(q, k, v, o, dO, p, st);
+      return launch_bwd<DkdvD64, DqD64>(q, k, v, o, dO, p, st);
     case 96:
     case 128: return launch_bwd<DkdvD128, DqD128>(q, k, v, o, dO, p, st);
     default: return launch_bwd<DkdvD256, DqD256>(q, k, v, o, dO, p, st);
@@ -892,7 +945,7 @@ fa_status fa_fwd_host(const void* q_host, const void* k_host, const void* v_host
 // ------------------------------------------------------------------ FP8 backward
 size_t fa_bwd_fp8_workspace_size(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
-  return 3 * fp8_bwd_tensor_bytes(B, H, N, d) + workspace_bytes(B, H, N);
+  return 3 * fp8_bwd_tensor_bytes(B, H, N, d) + bwd_workspace_need(B, H, N, d);
 }
 
 fa_status fa_bwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,

@@ -21,6 +21,14 @@
 // Splitting dQ into its own pass costs a second recompute of S and dP but needs
 // no fp32 atomics and is deterministic.
 //
+// At d = 64 (tensor memory has room there) the dK/dV pass also produces dQ:
+//   dQ_i += dS_i K                                      (tensor core, A = dS from smem)
+// accumulated in fp32 in the caller's workspace by TMA reduce-adds (each compute warp
+// stages its 32 x 32 block in shared memory), the sums zeroed by pass 1;
+// a fourth kernel, fa_bwd_dq_convert, writes dQ = scale dQ_acc in bf16, and pass 3 is
+// not run.  This is the pages' single-pass order (FA2: dQ accumulated while dK and dV
+// are built); the fp32 sums' order, and so dQ's last bits, vary from run to run.
+//
 // Roles in kernels 2 and 3: warps 0..7 elementwise work (two warps per TMEM lane
 // quadrant, each on half of the streamed tile's columns), warp 8 TMA producer, warp 9
 // MMA issuer (one elected lane issues; owns tensor memory).
@@ -43,6 +51,7 @@ struct BwdParams {
   float scale;
   const float* lse;      // [BH, N]
   const float* drow;     // D_i workspace [BH, N]
+  float* dq_acc;         // fused d = 64 dK/dV pass: fp32 [BH, N, 64] dQ sums, zeroed by pass 1
   void* dq;              // bf16 [BH, N, D]
   void* dk;
   void* dv;
@@ -72,10 +81,13 @@ __device__ __forceinline__ void bwd_block_item(int block, int heads, int levels,
 // D_i = sum_c dO_ic * O_ic, fp32 accumulation of the bf16 products.  A row of D
 // elements is D/8 16-byte pieces; TPR threads (a power of two) share a row, PER pieces
 // each: D = 64 -> 8 x 1, 128 -> 16 x 1, 256 -> 32 x 1, 96 -> 4 x 3, 192 -> 8 x 3.
+// With dq_acc (rows of D fp32 values, D = 64 only) the pass also zeroes each row's dQ
+// accumulator.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_rowdot(const __nv_bfloat16* __restrict__ o,
                                                      const __nv_bfloat16* __restrict__ dout,
-                                                     float* __restrict__ drow, long long rows) {
+                                                     float* __restrict__ drow, long long rows,
+                                                     float* __restrict__ dq_acc) {
   constexpr int PIECES = D / 8;
   constexpr int PER = (PIECES % 3 == 0) ? 3 : 1;   // pieces per thread
   constexpr int TPR = PIECES / PER;                  // threads per row
@@ -102,6 +114,31 @@ __global__ void __launch_bounds__(256) fa_bwd_rowdot(const __nv_bfloat16* __rest
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (sub == 0) drow[r] = acc;
+    if (dq_acc != nullptr) {
+      float4* z = reinterpret_cast<float4*>(dq_acc + r * D);
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        z[2 * (sub * PER + u)] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[2 * (sub * PER + u) + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------------- 4. dQ (fused)
+// dQ = scale * dQ_acc -> bf16, eight values per thread step (rows of 64, stored = kernel
+// head dim).  A programmatic dependent of the dK/dV pass: waits for all its sums.
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert(const float* __restrict__ acc,
+                                                         __nv_bfloat16* __restrict__ dq,
+                                                         long long n8, float scale) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * 256) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    reinterpret_cast<uint4*>(dq)[i] =
+        make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                   pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
   }
 }
 
@@ -122,7 +159,8 @@ __global__ void __launch_bounds__(256) fa_bwd_rowdot(const __nv_bfloat16* __rest
 // quadrant, each owning half of the BMQ query columns (P needs no row reduction, so
 // the halves never talk to each other).  Each half writes its bf16 P^T / dS^T into
 // the first half of its own column range.
-template <int D_, int DH_, int BMQ_, int QST_, int OST_, int SB_, int DB_, int EMU_ = 1>
+template <int D_, int DH_, int BMQ_, int QST_, int OST_, int SB_, int DB_, int EMU_ = 1,
+          bool FUSEDQ_ = false>
 struct DkdvCfg {
   static constexpr int D = D_;          // head dim (contraction of S^T and dP^T)
   static constexpr int DH = DH_;        // columns of dK/dV this CTA produces
@@ -147,13 +185,28 @@ struct DkdvCfg {
   // D_i by one step
   static constexpr int DDR = OST + 1;
   static constexpr int SMEM_DD = SMEM_LSE + QST * BMQ * 4;        // [DDR][BMQ] fp32
-  static constexpr int SMEM_BAR = SMEM_DD + DDR * BMQ * 4;
+  // Fused dQ (d = 64): dS^T also goes to shared memory in bf16, as two 128-byte
+  // swizzled boxes of 64 query columns x BN key rows.  Read column-wise, that is the
+  // A operand (MN-major) of dQ_i = dS_i K; K's resident tile is its B operand
+  // (MN-major, like V in the forward's P V).  dQ_i lands in the middle BMQ/2 columns
+  // of the step's S^T buffer: the halves' packed P^T sit at its two ends (PACK_HI).
+  static constexpr bool FUSEDQ = FUSEDQ_;
+  static constexpr int SMEM_DS =
+      FUSEDQ ? (SMEM_DD + DDR * BMQ * 4 + 1023) / 1024 * 1024 : SMEM_DD + DDR * BMQ * 4;
+  static constexpr int DS_BOX = BN * 128;                 // one box of 64 query columns
+  // and one 4 KB staging block per compute warp for its dQ reduce-add (32 rows x 32
+  // fp32, 128-byte swizzled)
+  static constexpr int SMEM_DQ = SMEM_DS + (FUSEDQ ? BN * BMQ * 2 : 0);
+  static constexpr int SMEM_BAR = SMEM_DQ + (FUSEDQ ? 8 * 4096 : 0);
+  static constexpr int PACK_HI = FUSEDQ ? BMQ - BMQ / 4 : BMQ / 2;
+  static constexpr int TM_DQ_OFF = BMQ / 4;
   static constexpr int B_KV = 0, B_ACC = 1, B_DRAIN = 2,
                        B_SFULL = 3, B_P = 3 + SB,                   // + buffer
                        B_DPFULL = 3 + 2 * SB, B_DS = 3 + 2 * SB + DB,
                        B_QFULL = 3 + 2 * SB + 2 * DB, B_QEMPTY = B_QFULL + QST,
                        B_OFULL = B_QEMPTY + QST, B_OEMPTY = B_OFULL + OST,
-                       NBARS = B_OEMPTY + OST;
+                       B_DQFULL = B_OEMPTY + OST, B_DQFREE = B_DQFULL + 1,
+                       NBARS = B_OEMPTY + OST + (FUSEDQ ? 2 : 0);
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
   static constexpr int TM_ST = 0;                        // + b * BMQ
@@ -166,6 +219,8 @@ struct DkdvCfg {
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(BMQ % 64 == 0 && DH % 64 == 0 && CH % 32 == 0, "box and TMEM chunk sizes");
   static_assert(SB >= 1 && SB <= 2 && DB >= 1 && DB <= 2, "one or two buffers");
+  static_assert(!FUSEDQ || (D == 64 && DH == 64 && BMQ == 128 && SB == 2 && DB == 1),
+                "fused dQ: d = 64, 128-row query tiles, two S^T buffers, one dP^T buffer");
 };
 
 template <class C>
@@ -176,10 +231,12 @@ __device__ __forceinline__ void dkdv_q_range(const BwdParams& p, int kt, int& i0
 
 // A = (BMQ x 128)^T operand kb (16 query columns) of the bf16 tile written over a
 // BMQ-column fp32 buffer: half h of the columns keeps its values in its own range.
-template <int BMQ>
+// The second half's values start at column HI (BMQ / 2: each half at the start of
+// its own range).
+template <int BMQ, int HI = BMQ / 2>
 __device__ __forceinline__ uint32_t half_packed_col(int kb) {
   constexpr int KB_H = BMQ / 2 / 16;      // 16-column blocks per half
-  return (kb / KB_H) * (BMQ / 2) + (kb % KB_H) * 8;
+  return (kb / KB_H) * HI + (kb % KB_H) * 8;
 }
 
 // 2^x of an even-length row segment into `pr`: EMU of every 4 pairs on the FMA pipe,
@@ -222,7 +279,7 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     fa_bwd_dkdv(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                const BwdParams p) {
+                const __grid_constant__ CUtensorMap tdq, const BwdParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ uint8_t smem_raw[];
@@ -255,7 +312,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i) {
-      const bool warps8 = (i >= C::B_P && i < C::B_P + C::SB) || (i >= C::B_DS && i < C::B_DS + C::DB);
+      const bool warps8 = (i >= C::B_P && i < C::B_P + C::SB) || (i >= C::B_DS && i < C::B_DS + C::DB) ||
+                          (C::FUSEDQ && i == C::B_DQFREE);
       mbar_init(bar(i), warps8 ? 8u : 1u);                  // 8 compute warps arrive
     }
     *abort_flag = 0;
@@ -395,7 +453,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // Tile st+1's products go ahead of tile st's gradient products when they have a
     // buffer of their own and their operand tile can already be resident (a second
     // ring slot); otherwise they follow them.
-    constexpr bool EARLY_S = C::SB == 2 && C::QST >= 2;
+    // fused dQ: S^T(st+1) goes into the buffer that holds dQ(st-1), once the compute
+    // warps have drained it (after dV(st), below)
+    constexpr bool EARLY_S = C::SB == 2 && C::QST >= 2 && !C::FUSEDQ;
     constexpr bool EARLY_DP = EARLY_S && C::DB == 2 && C::OST >= 2;
     for (int st = 0; st < nsteps && ok; ++st) {
       const int nx = st + 1;
@@ -408,10 +468,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const uint32_t stb = tmem + C::TM_ST + (st % C::SB) * C::BMQ;
 #pragma unroll
       for (int kb = 0; kb < C::BMQ / 16; ++kb)
-        umma_ts_elect(false, tmem + C::TM_DV, stb + half_packed_col<C::BMQ>(kb),
+        umma_ts_elect(false, tmem + C::TM_DV, stb + half_packed_col<C::BMQ, C::PACK_HI>(kb),
                       sdesc_sw128(dobuf(st) + hbox * C::BMQ * 128 + kb * 16 * 128, C::BMQ * 128, 1024),
                       ID_G, (st > 0 || kb > 0) ? 1u : 0u);
       tc_commit_elect(bar(C::B_OEMPTY + st % C::OST));     // dP^T(st) and dV(st) read dO(st)
+      if constexpr (C::FUSEDQ) {
+        if (nx < nsteps) {
+          if (st >= 1 &&
+              !(ok = mbar_wait_warp(bar(C::B_DQFREE), (st - 1) & 1, wc, kSiteDqDone)))
+            break;
+          if (!(ok = issue_st(nx))) break;
+        }
+      }
       // dK += dS^T Q[:, part]   (A = dS^T bf16 in TMEM over the dP^T columns)
       if (!(ok = mbar_wait_warp(bar(C::B_DS + st % C::DB), (st / C::DB) & 1, wc, kSiteDsFull))) break;
       tc_fence_after();
@@ -422,9 +490,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       sdesc_sw128(qbuf(st) + hbox * C::BMQ * 128 + kb * 16 * 128, C::BMQ * 128, 1024),
                       ID_G, (st > 0 || kb > 0) ? 1u : 0u);
       tc_commit_elect(bar(C::B_QEMPTY + st % C::QST));     // S^T(st) and dK(st) read Q(st)
+      if constexpr (C::FUSEDQ) {
+        // dQ(st) = dS(st) K: A = dS from shared memory (MN-major), B = K (MN-major)
+        constexpr uint32_t ID_Q = idesc_bf16_amn(128, C::D, true);
+        const uint32_t dqt = tmem + C::TM_ST + (st % C::SB) * C::BMQ + C::TM_DQ_OFF;
+#pragma unroll
+        for (int kb = 0; kb < C::BN / 16; ++kb)
+          umma_ss_elect(false, dqt, sdesc_sw128(sbase + C::SMEM_DS + kb * 16 * 128, C::DS_BOX, 1024),
+                        sdesc_sw128(sbase + C::SMEM_K + kb * 16 * 128, C::BN * 128, 1024), ID_Q,
+                        kb > 0 ? 1u : 0u);
+        tc_commit_elect(bar(C::B_DQFULL));
+      }
       // the next tile's remaining products go after this tile's readers
       if (nx < nsteps) {
-        if (!EARLY_S && !(ok = issue_st(nx))) break;
+        if (!EARLY_S && !C::FUSEDQ && !(ok = issue_st(nx))) break;
         if (!EARLY_DP && !(ok = issue_dpt(nx))) break;
       }
     }
@@ -440,6 +519,34 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t lb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float sl2 = p.scale * LOG2E;
     bool ok = true;
+    // fused dQ: add dQ(sp) (this warp's lane quadrant of query rows, its half of the
+    // columns) into the fp32 accumulator, then free its tensor-memory columns
+    auto drain_dq = [&](int sp) -> bool {
+      if (!mbar_wait(bar(C::B_DQFULL), sp & 1, wc, kSiteDqDone)) return false;
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld32(lb + C::TM_ST + (sp % C::SB) * C::BMQ + C::TM_DQ_OFF + half * 32, r);
+      tmem_ld_wait(r);
+      tc_fence_before();
+      mbar_arrive_warp(bar(C::B_DQFREE));          // the columns are free once loaded
+      // staging block: row `lane`, 16-byte chunk c at position c ^ (lane & 7); the
+      // previous reduce-add from it has read it (one step ago)
+      const uint32_t stg = sbase + C::SMEM_DQ + warp * 4096;
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(stg + lane * 128 + ((c ^ (lane & 7)) << 4), r[4 * c], r[4 * c + 1], r[4 * c + 2],
+                     r[4 * c + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int y = q_tile(sp) * C::BMQ + quad * 32;   // first query row of the block
+      if (lane == 0 && y < p.N) {                        // rows past N are clipped
+        tma_reduce_add_3d(&tdq, stg, half * 32, y, q_head(sp));
+        bulk_commit();
+      }
+      return true;
+    };
     for (int st = 0; st < nsteps && ok; ++st) {
       const int qi = q_tile(st);
       const int c_first = qi * C::BMQ + half * C::CH;      // first query of this half
@@ -451,6 +558,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_fence_after();
       const float* ls = lse_s + (st % C::QST) * C::BMQ + half * C::CH;
       const uint32_t stc = lb + C::TM_ST + (st % C::SB) * C::BMQ + half * C::CH;
+      const uint32_t stp = lb + C::TM_ST + (st % C::SB) * C::BMQ + half * C::PACK_HI;
       // P^T row segment, zero where the query may not see this key
       float pr[C::CH];
       {
@@ -478,13 +586,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < C::CH / 2; ++i) w[i] = pack_bf16x2(pr[2 * i], pr[2 * i + 1]);
         if constexpr (C::CH == 64)
-          tmem_st32(stc, w);
+          tmem_st32(stp, w);
         else
-          tmem_st16(stc, w);
+          tmem_st16(stp, w);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive_warp(bar(C::B_P + st % C::SB));
+      if constexpr (C::FUSEDQ) {
+        // dQ(st-1) is done by now; its drain also frees the shared dS tile for this step
+        if (st > 0 && !(ok = drain_dq(st - 1))) break;
+      }
       // dS^T row segment = P^T (dP^T - D_q), bf16 over this half's dP^T columns
       if (!(ok = mbar_wait(bar(C::B_DPFULL + st % C::DB), (st / C::DB) & 1, wc, kSiteSFull))) break;
       tc_fence_after();
@@ -512,10 +624,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tmem_st32(dpc, w);
         else
           tmem_st16(dpc, w);
+        if constexpr (C::FUSEDQ) {
+          // the same row of dS^T into shared memory: box `half`, row `row`, 16-byte
+          // chunk c of 8 queries at chunk position c ^ (row & 7) (128-byte swizzle)
+          const uint32_t ds_row = sbase + C::SMEM_DS + half * C::DS_BOX + row * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(ds_row + ((c ^ (row & 7)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
+                         w[4 * c + 3]);
+          fence_proxy_async_smem();
+        }
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive_warp(bar(C::B_DS + st % C::DB));
+    }
+    if constexpr (C::FUSEDQ) {
+      if (ok && nsteps > 0) ok = drain_dq(nsteps - 1);
     }
     // epilogue: dV and scale*dK -> bf16 global, this half's DH/2 columns of the row
     if (ok && mbar_wait(bar(C::B_ACC), 0, wc, kSiteDqDone)) {
@@ -547,6 +672,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
         }
       }
+    }
+    // fused dQ: this warp's reduce-adds complete before its shared memory goes away
+    if constexpr (C::FUSEDQ) {
+      if (lane == 0) bulk_wait_all();
     }
   }
 

@@ -126,8 +126,9 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
                      int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
- * fa_bwd_workspace_size — bytes of device workspace fa_bwd needs for these sizes
- * (fp32 D_i = sum_c dO_ic O_ic for every row, 256-byte aligned).  0 when B*H*N == 0.
+ * fa_bwd_workspace_size — bytes of device workspace fa_bwd needs for these sizes:
+ * fp32 D_i = sum_c dO_ic O_ic for every row, 256-byte aligned, and at d = 64 also
+ * the fp32 dQ sums [B,H,N,64] (256-byte aligned).  0 when B*H*N == 0.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -144,9 +145,13 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *   workspace        scratch device memory of >= fa_bwd_workspace_size() bytes,
  *                    owned by the caller; contents on entry are ignored.
  * Launches, in stream order: the D_i row-sum pass, the dK/dV pass (one CTA per
- * key tile) and the dQ pass (one CTA per query tile).  Deterministic: no
- * atomics.  Errors as fa_fwd, plus FA_ERR_INVALID_ARG when the workspace is
- * too small.
+ * key tile) and the dQ pass (one CTA per query tile); deterministic.  At d = 64
+ * the dK/dV pass also forms dQ (the pages' FA2 order): the row-sum pass zeroes
+ * fp32 dQ sums in the workspace, the dK/dV CTAs add their key tile's share with
+ * TMA reduce-adds, and a last pass writes dQ = scale * sums in bf16.  There dK
+ * and dV repeat bit for bit, dQ to within its last bits (the order of the fp32
+ * additions varies).  Errors as fa_fwd, plus FA_ERR_INVALID_ARG when the
+ * workspace is too small.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                  const float* lse, void* dq, void* dk, void* dv,
@@ -190,7 +195,8 @@ fa_status fa_bwd_fp8(const void* q8, const void* k8, const void* v8,
  * host program that owns every byte of device memory through its own pool, or a
  * latency-critical path where cudaMalloc's implicit device-wide synchronisation
  * is not acceptable.  This entry point takes the same inputs and outputs as
- * fa_bwd and gives the same results, but keeps the per-row D_i scratch in a fixed
+ * fa_bwd and gives the same results (at d = 64 through the separate dQ pass, which
+ * needs no dQ sums), but keeps the per-row D_i scratch in a fixed
  * array inside the library (FA_BWD_NOALLOC_MAX_ROWS fp32 values = 8 MiB, held on
  * every GPU that loads the library until the process exits).  It calls no
  * cudaMalloc, cudaFree or other allocating routine.

@@ -100,6 +100,21 @@ def test_bwd_is_deterministic(fa):
     assert all(torch.equal(a, b) for a, b in zip(g1, g2))
 
 
+def test_bwd_d64_repeatability(fa):
+    """At d = 64 dQ is summed over key tiles by fp32 reduce-adds in whatever order the
+    CTAs reach them, so only its last bits may differ between runs; dK and dV, which
+    each CTA owns, repeat exactly."""
+    w = workloads.make_small(2, 3, 1000, 64, True, seed=12, backward=True)
+    q, k, v, do = (t.cuda() for t in workloads.make_bf16_inputs(w))
+    o, lse = fa.attention_forward(q, k, v, causal=True)
+    dq1, dk1, dv1 = fa.attention_backward(q, k, v, o, do, lse, causal=True)
+    dq2, dk2, dv2 = fa.attention_backward(q, k, v, o, do, lse, causal=True)
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    diff = (dq1.float() - dq2.float()).abs()
+    # at most one bf16 rounding step of the value
+    assert bool((diff <= dq1.float().abs() * 2.0 ** -7 + 1e-30).all())
+
+
 def test_bwd_workspace_too_small_raises(fa):
     q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device="cuda")
     lse = torch.zeros(1, 1, 128, dtype=torch.float32, device="cuda")
