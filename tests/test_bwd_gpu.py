@@ -26,6 +26,7 @@ def run_fwd_bwd(fa, q, k, v, do, causal, scale):
 
 SMALL = [
     (1, 2, 128, 64, False), (1, 2, 256, 64, True), (2, 2, 500, 64, True), (1, 2, 640, 64, False),
+    (2, 3, 1000, 64, True),
     (1, 2, 384, 128, True), (2, 1, 700, 128, False),
     (1, 2, 256, 256, True), (1, 1, 330, 256, False),
     (1, 1, 1, 64, True), (1, 1, 50, 128, True),

@@ -46,7 +46,7 @@ def test_gqa_forward_matches_oracle(fa, B, Hq, Hkv, N, d, causal):
 
 BWD = [
     (1, 4, 2, 300, 64, True), (1, 8, 1, 257, 128, False), (1, 4, 2, 200, 256, True),
-    (2, 6, 3, 400, 128, True),
+    (2, 6, 3, 400, 128, True), (2, 4, 1, 513, 64, False),
 ]
 
 
