@@ -16,7 +16,6 @@
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd_pp.cuh"
-#include "fa_fwd_ws.cuh"
 #include "fa_decode.cuh"
 #include "fa_dequant.cuh"
 #include "sm100_ptx.cuh"
@@ -262,33 +261,6 @@ fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p
   return FA_OK;
 }
 
-// One query tile per CTA, split softmax, two output accumulators (fa_fwd_ws.cuh).
-template <class C>
-fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p,
-                        cudaStream_t stream) {
-  DeviceInfo* di = nullptr;
-  if (fa_status s = device_info(&di)) return s;
-  CUtensorMap mq, mk, mv;
-  if (fa_status s = make_map(&mq, q, C::FP8, p.ld, p.N, p.BH, C::BM)) return s;
-  if (fa_status s = make_map(&mk, k, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
-  if (fa_status s = make_map(&mv, v, C::FP8, p.ld, p.N, p.BH / p.g, C::BN)) return s;
-  auto kern = fa_fwd_ws_kernel<C>;
-  if (fa_status s = prepare_kernel<C>(kern, C::SMEM_ALLOC)) return s;
-  p.n_qt = (p.N + C::BM - 1) / C::BM;
-  p.n_kt = (p.N + C::BN - 1) / C::BN;
-  p.n_st = (p.N + 127) / 128;
-  p.total_items = p.BH * p.n_qt;
-  p.group_heads = causal_group_heads(p.BH, 2ll * p.N * C::D * C::ELEM);
-  p.status = di->status;
-  p.timeout_ns = kWaitTimeoutNs;
-  p.sched = sched_counter(di, stream);
-  const int grid = p.total_items < di->sms ? p.total_items : di->sms;
-  kern<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
-  return FA_OK;
-}
-
 // Tuning knobs (compile-time): software-exp2 share, pipeline depth, kernel family.
 // software-exp2 share (quarters of the exponentials) per problem class, measured: the
 // two-tile kernel wants 1 at d = 64 and FP8 (2 and 3 were slower) and none at bf16
@@ -310,20 +282,11 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #ifndef FA_FWD_D256_TAU
 #define FA_FWD_D256_TAU 8
 #endif
-#ifndef FA_FWD_WS_INDEP
-#define FA_FWD_WS_INDEP 1
-#endif
-#ifndef FA_FWD_WS_SPLIT
-#define FA_FWD_WS_SPLIT 0
-#endif
 #ifndef FA_FWD_D128_KST
 #define FA_FWD_D128_KST 2
 #endif
 #ifndef FA_FWD_D128_VST
 #define FA_FWD_D128_VST 2
-#endif
-#ifndef FA_FWD_WS_TAU
-#define FA_FWD_WS_TAU 8
 #endif
 // two-tile kernel, bf16: rescale threshold (log2 units) with the compensated row sum
 // (measured: +6.7 % on N(0,1) inputs at N = 32768, +1 % at d = 64, neutral on the
@@ -338,8 +301,7 @@ fa_status launch_fwd_ws(const void* q, const void* k, const void* v, FwdParams p
 #define FA_FWD_EXPH 0
 #endif
 // Kernel family per problem class (measured fastest on the causal N = 4096 workloads):
-// 0 = one query tile per CTA (fa_fwd.cuh), 1 = two query tiles (fa_fwd_pp.cuh),
-// 2 = split softmax (fa_fwd_ws.cuh).
+// 0 = one query tile per CTA (fa_fwd.cuh), 1 = two query tiles (fa_fwd_pp.cuh).
 #ifndef FA_FWD_D64_KIND
 #define FA_FWD_D64_KIND 1
 #endif
@@ -358,15 +320,11 @@ struct FwdPick {
   static constexpr int VST = kWide ? FA_FWD_D128_VST : 4;
   using Cfg = std::conditional_t<
       KIND == 0, FwdCfg<D, 128, kWide ? 3 : 4, kWide ? 2 : 4, FP8, EMU>,
-      std::conditional_t<
-          KIND == 1, PPCfg<D, KST, VST, FP8, EMU, FA_FWD_TAU, FA_FWD_EXPH, FA_FWD_PP_COMP != 0>,
-          WSCfg<D, KST, VST, FP8, EMU, EMU, FA_FWD_WS_SPLIT != 0, FA_FWD_WS_INDEP != 0,
-                FA_FWD_WS_TAU>>>;
-  static_assert(KIND >= 0 && KIND <= 2, "kernel family 0, 1 or 2");
+      PPCfg<D, KST, VST, FP8, EMU, FA_FWD_TAU, FA_FWD_EXPH, FA_FWD_PP_COMP != 0>>;
+  static_assert(KIND == 0 || KIND == 1, "kernel family 0 or 1");
   static const char* name() {
     static const std::string n = [] {
-      static const char* fam[] = {"fa_fwd_kernel<FwdCfg", "fa_fwd_pp_kernel<PPCfg",
-                                  "fa_fwd_ws_kernel<WSCfg"};
+      static const char* fam[] = {"fa_fwd_kernel<FwdCfg", "fa_fwd_pp_kernel<PPCfg"};
       char buf[128];
       std::snprintf(buf, sizeof buf, "%s<%d,KST%d,VST%d,%s>>", fam[KIND], D, Cfg::KST, Cfg::VST,
                     FP8 ? "e4m3" : "bf16");
@@ -378,10 +336,8 @@ struct FwdPick {
                           cudaStream_t st) {
     if constexpr (KIND == 0)
       return launch_fwd<Cfg>(q, k, v, p, st);
-    else if constexpr (KIND == 1)
-      return launch_fwd_pp<Cfg>(q, k, v, p, st);
     else
-      return launch_fwd_ws<Cfg>(q, k, v, p, st);
+      return launch_fwd_pp<Cfg>(q, k, v, p, st);
   }
 };
 using FwdD64 = FwdPick<FA_FWD_D64_KIND, 64, false, FA_FWD_D64_EMU>;

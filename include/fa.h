@@ -295,7 +295,7 @@ int fa_version(void);
 /*
  * fa_fwd_kernel_name — name of the forward kernel that fa_fwd (fp8 = 0) or
  * fa_fwd_fp8 (fp8 != 0) launches for head dimension `head_dim`, with its
- * tile configuration, e.g. "fa_fwd_ws_kernel<WSCfg<128,KST2,VST2,bf16>>".  The
+ * tile configuration, e.g. "fa_fwd_pp_kernel<PPCfg<128,KST2,VST2,bf16>>".  The
  * string is static and owned by the library.  Returns NULL for an unsupported
  * head dimension.  Host only; launches nothing.
  */
