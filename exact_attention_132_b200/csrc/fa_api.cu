@@ -62,7 +62,7 @@ struct DeviceInfo {
   std::mutex host_mu;
   bool host_ready = false;
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
-  cudaEvent_t host_ev[64] = {};   // >= 1 + 3 * kHostChunks
+  cudaEvent_t host_ev[128] = {};   // >= 1 + 3 * kHostChunks
   cudaStream_t sched_stream[kSchedSlots] = {};
   int sched_used = 0;
 };
@@ -515,8 +515,11 @@ size_t fp8_bwd_tensor_bytes(int B, int H, int N, int d) {
 // more chunks shorten the copy-in before the first kernel and the copy-out after the last),
 // each staged in one of two device slots.  A slot holds Q, K, V, O (bf16) and LSE (fp32)
 // of `hc` heads, each part 256-byte aligned.
-constexpr int kHostChunks = 16;
-static_assert(1 + 3 * kHostChunks <= 64, "host pipeline event pool");
+#ifndef FA_HOST_CHUNKS
+#define FA_HOST_CHUNKS 16
+#endif
+constexpr int kHostChunks = FA_HOST_CHUNKS;
+static_assert(1 + 3 * kHostChunks <= 128, "host pipeline event pool");
 int host_chunk_heads(int BH) {
   const int nc = BH < kHostChunks ? BH : kHostChunks;
   return (BH + nc - 1) / nc;
@@ -834,7 +837,7 @@ fa_status fa_fwd_host(const void* q_host, const void* k_host, const void* v_host
   if (!di->host_ready) {
     cudaError_t e = cudaStreamCreateWithFlags(&di->copy_in, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&di->copy_out, cudaStreamNonBlocking);
-    for (int i = 0; e == cudaSuccess && i < 64; ++i)
+    for (int i = 0; e == cudaSuccess && i < 1 + 3 * kHostChunks; ++i)
       e = cudaEventCreateWithFlags(&di->host_ev[i], cudaEventDisableTiming);
     if (e != cudaSuccess) return cuda_fail(e, "host pipeline setup");
     di->host_ready = true;

@@ -86,3 +86,37 @@ def test_forward_and_decode_replay_from_a_cuda_graph(fa):
         assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
         assert torch.equal(od, od_ref) and torch.equal(ld, ld_ref)
     assert fa.fa_get_device_status() == 0
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_replays_from_a_cuda_graph(fa, d):
+    """The backward's chained launches (programmatic dependents; at d = 64 the zeroing
+    row-dot pass, the dK/dV pass with its dQ reduce-adds and the convert pass) captured
+    once and replayed: every replay starts from zeroed dQ sums and matches eager runs."""
+    w, (q, k, v) = _inputs(1, 4, 700, d, True, seed=40 + d)
+    do = torch.randn_like(q.float()).to(torch.bfloat16)
+    o, lse = fa.attention_forward(q, k, v, causal=True, scale=w.sm_scale)
+    ref = fa.attention_backward(q, k, v, o, do, lse, causal=True, scale=w.sm_scale)
+    torch.cuda.synchronize()
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = torch.empty(fa.fa_bwd_workspace_size(1, 4, 700, d), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale=w.sm_scale, causal=True, stream=s)
+    s.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale=w.sm_scale, causal=True, stream=s)
+    for _ in range(4):
+        dq.zero_()
+        dk.zero_()
+        dv.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
+        if d == 64:   # dQ sums in varying order: equal to within its last bits
+            diff = (dq.float() - ref[0].float()).abs()
+            assert bool((diff <= ref[0].float().abs() * 2.0 ** -7 + 1e-30).all())
+        else:
+            assert torch.equal(dq, ref[0])
+    assert fa.fa_get_device_status() == 0
