@@ -346,9 +346,10 @@ using FwdF8D128 = FwdPick<FA_FWD_F8_KIND, 128, true, FA_FWD_F8_EMU>;
 using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_D256_EMU, FA_FWD_D256_TAU>;
 using FwdF8D256 = FwdCfg<256, 128, 3, 2, true, FA_FWD_F8_EMU>;
 
-// backward software-exp2 share: a quarter at d = 64 and 128, none at d = 256 (measured)
+// backward software-exp2 share: none (measured: at d = 64 with dQ formed in the dK/dV pass
+// 671 against 658 TFLOP/s with a quarter, a half 649; at d = 128 750 either way)
 #ifndef FA_BWD_EMU
-#define FA_BWD_EMU 1
+#define FA_BWD_EMU 0
 #endif
 #ifndef FA_BWD_D256_EMU
 #define FA_BWD_D256_EMU 0
