@@ -282,6 +282,10 @@ fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p
 #ifndef FA_FWD_D256_TAU
 #define FA_FWD_D256_TAU 8
 #endif
+// ring depth of the two-tile kernel at d = 64 and FP8 (K and V each)
+#ifndef FA_FWD_NARROW_ST
+#define FA_FWD_NARROW_ST 4
+#endif
 #ifndef FA_FWD_D128_KST
 #define FA_FWD_D128_KST 2
 #endif
@@ -316,8 +320,8 @@ template <int KIND, int D, bool FP8, int EMU>
 struct FwdPick {
   // stage depths: deep rings where shared memory allows, 2 + 2 for bf16 d = 128
   static constexpr bool kWide = (D == 128 && !FP8);
-  static constexpr int KST = kWide ? FA_FWD_D128_KST : 4;
-  static constexpr int VST = kWide ? FA_FWD_D128_VST : 4;
+  static constexpr int KST = kWide ? FA_FWD_D128_KST : FA_FWD_NARROW_ST;
+  static constexpr int VST = kWide ? FA_FWD_D128_VST : FA_FWD_NARROW_ST;
   using Cfg = std::conditional_t<
       KIND == 0, FwdCfg<D, 128, kWide ? 3 : 4, kWide ? 2 : 4, FP8, EMU>,
       PPCfg<D, KST, VST, FP8, EMU, FA_FWD_TAU, FA_FWD_EXPH, FA_FWD_PP_COMP != 0>>;
