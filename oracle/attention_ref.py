@@ -17,7 +17,7 @@ fused method reaches this same result up to floating-point rounding
 softmaxの再スケール; wiki, section オンラインSoftmax計算), so the definition is
 the oracle.
 
-Readings of points the pages leave open (each also listed in the design doc):
+Readings of points the pages leave open:
 
 * causal = lower triangular, key j visible to query i iff j <= i (the pages say
   only "lower-triangular mask", mypcrig.com post, section "FA2 の改善").
