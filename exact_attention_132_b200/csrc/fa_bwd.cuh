@@ -26,8 +26,8 @@
 // accumulated in fp32 in the caller's workspace by TMA reduce-adds (each compute warp
 // stages its 32 x 32 block in shared memory), the sums zeroed by pass 1;
 // a fourth kernel, fa_bwd_dq_convert, writes dQ = scale dQ_acc in bf16, and pass 3 is
-// not run.  This is the pages' single-pass order (FA2: dQ accumulated while dK and dV
-// are built); the fp32 sums' order, and so dQ's last bits, vary from run to run.
+// not run (a build choice: the pages give only the recompute).  The fp32 sums' order,
+// and so dQ's last bits, vary from run to run.
 //
 // Roles in kernels 2 and 3: warps 0..7 elementwise work (two warps per TMEM lane
 // quadrant, each on half of the streamed tile's columns), warp 8 TMA producer, warp 9

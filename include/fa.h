@@ -146,7 +146,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *                    owned by the caller; contents on entry are ignored.
  * Launches, in stream order: the D_i row-sum pass, the dK/dV pass (one CTA per
  * key tile) and the dQ pass (one CTA per query tile); deterministic.  At d = 64
- * the dK/dV pass also forms dQ (the pages' FA2 order): the row-sum pass zeroes
+ * the dK/dV pass also forms dQ (a build choice): the row-sum pass zeroes
  * fp32 dQ sums in the workspace, the dK/dV CTAs add their key tile's share with
  * TMA reduce-adds, and a last pass writes dQ = scale * sums in bf16.  There dK
  * and dV repeat bit for bit, dQ to within its last bits (the order of the fp32
