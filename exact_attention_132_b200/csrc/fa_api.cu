@@ -372,7 +372,7 @@ using DkdvD64F =
 using DkdvD128 = DkdvCfg<128, 128, 64, 3, 3, 2, 2, FA_BWD_EMU>;
 using DkdvD256 = DkdvCfg<256, 128, 64, 2, 1, 2, 2, FA_BWD_D256_EMU>;
 using DqD64 = DqCfg<64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU>;
-using DqD128 = DqCfg<128, 128, 2, 2, 2, 1, FA_BWD_EMU>;
+using DqD128 = DqCfg<128, 128, 3, 2, 2, 1, FA_BWD_EMU>;
 using DqD256 = DqCfg<256, 64, 2, 1, 2, 2, FA_BWD_D256_EMU>;
 
 // Launch `kern` as a programmatic dependent of the previous kernel in `stream`: it may
