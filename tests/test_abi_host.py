@@ -156,3 +156,29 @@ def test_decode_argument_errors_return_before_any_cuda_call():
     assert _dec(B=-1) == 1
     assert _dec(Nq=0) == 0 and _dec(B=0) == 0           # empty problems are no-ops
     assert fa.fa_decode_workspace_size(1, 6, 4, 1, 100, 128) == 0
+
+
+def test_noalloc_backward_argument_errors_return_before_any_cuda_call():
+    # the Python constant is the header's limit
+    hdr = open(os.path.join(ROOT, "include", "fa.h")).read()
+    m = re.search(r"#define\s+FA_BWD_NOALLOC_MAX_ROWS\s+\(1 << (\d+)\)", hdr)
+    assert m and fa.FA_BWD_NOALLOC_MAX_ROWS == 1 << int(m.group(1))
+    P = lambda x: ctypes.c_void_p(16 * x)
+    ptrs = [P(1)] * 9
+
+    def call(B=1, H=2, N=256, d=128, scale=0.125, ps=ptrs):
+        return fa.lib.fa_bwd_noalloc(*ps, B, H, N, d, scale, 1, None)
+
+    assert call(d=80) == fa.FA_ERR_UNSUPPORTED
+    assert call(N=-1) == fa.FA_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == fa.FA_ERR_INVALID_ARG
+    # one row past the fixed scratch, and exactly at it with a null pointer (so that the
+    # size check passes and the pointer check answers, still before any CUDA call)
+    H, N = 32, fa.FA_BWD_NOALLOC_MAX_ROWS // 32
+    assert call(B=1, H=H, N=N + 1) == fa.FA_ERR_INVALID_ARG
+    assert "exceeds the fixed scratch" in fa.fa_last_error_string()
+    nulls = ptrs[:6] + [None] + ptrs[7:]
+    assert call(B=1, H=H, N=N, ps=nulls) == fa.FA_ERR_INVALID_ARG
+    assert "dq" in fa.fa_last_error_string()
+    # empty problems launch nothing and touch no pointer
+    assert call(B=0, ps=[None] * 9) == fa.FA_OK
