@@ -156,6 +156,8 @@ def test_unmutated_decode_passes():
         assert chk(_dec_generic), chk.__name__
 
 
+# a mutant that masks every key of a row produces NaN rows on purpose
+@pytest.mark.filterwarnings("ignore:invalid value encountered:RuntimeWarning")
 @pytest.mark.parametrize("name", sorted(MUTANTS_DEC))
 def test_decode_mutant_is_caught(name):
     kw = MUTANTS_DEC[name]
