@@ -46,8 +46,8 @@ METRIC = "attention TFLOP/s fwd and fwd+bwd on 1 B200; % of dense BF16/FP8 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per launch of the headline forward kernel, from ncu's
-# dram__bytes_read.sum + dram__bytes_write.sum (profiles/
-# fa_fwd_d128_causal_B4H16N4096.md), keyed by a hash of the kernel sources and the
+# dram__bytes_read.sum + dram__bytes_write.sum in one capture of that kernel (the
+# summary under profiles/ gives the command), keyed by a hash of the kernel sources and the
 # launched kernel's name (which carries its tile configuration).  A changed kernel has
 # no entry and reports traffic = null.
 FWD_TRAFFIC_BYTES = {"ec7d2c01b8744ef8": 248_282_368}
@@ -251,11 +251,12 @@ def run_ours(args):
     extras = {}
     if not args.no_extras:
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        extras = run_extras(fa, dev, stream, max(3, min(args.steps, 10)), peak, hbm)
+        extras = run_extras(fa, dev, stream, max(20, min(args.steps, 100)), peak, hbm, local)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
+        cpu["sdpa_fp32_cpu"] = cpu_sdpa_figure()
 
     kname = fa.fa_fwd_kernel_name(w.d)
     line = {
@@ -298,11 +299,92 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def run_extras(fa, dev, stream, steps, peak, hbm_peak):
-    """fwd+bwd at the two backward workloads, the headline kernel at N=32768 and the FP8
-    forward; device-side seeded inputs."""
-    out = {}
+def timed_region(fn, steps, warmup, stream, gpu, min_ms=40.0):
+    """Time at least `steps` calls (more if needed so that the region lasts about `min_ms`,
+    long enough for the clock sampler) with CUDA events on `stream`, sampling the SM
+    clock and throttle reasons meanwhile.  Returns (total ms, per-call ms list, steps,
+    clocks)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    one = max(a.elapsed_time(b), 1e-3)
+    steps = max(steps, int(math.ceil(min_ms / one)))
+    clk = ClockSampler(gpu)
+    clk.start()
+    tot, per = time_steps(fn, steps, 0, stream)
+    return tot, per, steps, clk.stop()
+
+
+def roofline_obj(achieved, peak, unit, source, bound="tensor"):
+    return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "peak_source": source}
+
+
+def measure_fp8_peak(dev, gpu):
+    """Dense e4m3 matmul throughput: torch._scaled_mm on 8192^3 (2*N^3 FLOPs), best of 10
+    back-to-back launches, unit scales, bf16 output.  The FP8 counterpart of the bf16
+    matmul peak the headline is compared with."""
+    n = 8192
     gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    a = torch.randn((n, n), generator=gen, device=dev).to(torch.float8_e4m3fn)
+    bt = torch.randn((n, n), generator=gen, device=dev).to(torch.float8_e4m3fn)
+    one = torch.ones((), dtype=torch.float32, device=dev)
+    mm = lambda: torch._scaled_mm(a, bt.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    try:
+        for _ in range(3):
+            mm()
+        torch.cuda.synchronize()
+    except (RuntimeError, AttributeError) as e:   # no FP8 matmul in this torch build
+        return {"unavailable": str(e).splitlines()[0][:200]}
+    best = float("inf")
+    clk = ClockSampler(gpu)
+    clk.start()
+    for _ in range(10):
+        x = torch.cuda.Event(enable_timing=True)
+        y = torch.cuda.Event(enable_timing=True)
+        x.record()
+        mm()
+        y.record()
+        torch.cuda.synchronize()
+        best = min(best, x.elapsed_time(y))
+    c = clk.stop()
+    del a, bt
+    return {"tflops": round(2.0 * n ** 3 / (best * 1e-3) / 1e12, 1), "ms": round(best, 4),
+            "how": "torch._scaled_mm e4m3 x e4m3 -> bf16, 8192^3, best of 10", "clocks": c}
+
+
+def run_extras(fa, dev, stream, steps, peak, hbm_peak, gpu):
+    """The other workloads of the metric, each with its own clock record and roofline:
+    the small forward (latency), fwd+bwd at the two backward workloads, the headline
+    kernel at N=32768, decoding and the FP8 forward/backward (against a measured FP8
+    matmul peak).  Device-side seeded inputs."""
+    out = {}
+    src = "measured bf16 dense matmul (burst)"
+    gen = torch.Generator(device=dev)
+    # the small forward: 64 query tiles on 148 SMs, so latency-bound; reported, not graded
+    w = workloads.WORKLOADS["fwd_small"]
+    gen.manual_seed(w.seed)
+    shp = (w.B, w.H, w.N, w.d)
+    q, k, v = (torch.randn(shp, generator=gen, device=dev).to(torch.bfloat16) for _ in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty(shp[:3], dtype=torch.float32, device=dev)
+    tot, per, n_, clk = timed_region(
+        lambda: fa.fa_fwd(q, k, v, o, lse, scale=w.sm_scale, causal=True, stream=stream),
+        steps, 5, stream, gpu)
+    tf = w.fwd_flops() / (statistics.mean(per) * 1e-3) / 1e12
+    out["fwd_small"] = {"workload": "bf16 causal forward B=1 H=8 N=1024 d=64 scale=1/8",
+                        "steps": n_, "us_per_call": round(statistics.median(per) * 1e3, 2),
+                        "tflops_fwd": round(tf, 2),
+                        "note": "64 query tiles for 148 SMs: latency-bound, not graded",
+                        "roofline": roofline_obj(tf, peak, "TFLOP/s", src), "clocks": clk}
+    del q, k, v, o, lse
     for name in ("fwdbwd_d64", "fwdbwd_d256"):
         w = workloads.WORKLOADS[name]
         gen.manual_seed(w.seed)
@@ -322,17 +404,24 @@ def run_extras(fa, dev, stream, steps, peak, hbm_peak):
         def fwd_only():
             fa.fa_fwd(q, k, v, o, lse, scale=w.sm_scale, causal=w.causal, stream=stream)
 
-        tot, _ = time_steps(fb, steps, 2, stream)
-        ftot, _ = time_steps(fwd_only, steps, 2, stream)
+        tot, _, n_fb, clk = timed_region(fb, steps, 2, stream, gpu)
+        ftot, _, n_f, fclk = timed_region(fwd_only, steps, 2, stream, gpu)
         fl = w.fwd_flops() + w.bwd_flops()
+        ms_fb, ms_f = tot / n_fb, ftot / n_f
+        tf_fb = fl / (ms_fb * 1e-3) / 1e12
+        tf_f = w.fwd_flops() / (ms_f * 1e-3) / 1e12
+        tf_b = w.bwd_flops() / ((ms_fb - ms_f) * 1e-3) / 1e12 if ms_fb > ms_f else None
         out[name] = {"workload": f"B={w.B} H={w.H} N={w.N} d={w.d} "
                                  f"{'causal' if w.causal else 'non-causal'} fwd+bwd",
-                     "tflops_fwd_bwd": round(fl * steps / (tot * 1e-3) / 1e12, 2),
-                     "tflops_fwd": round(w.fwd_flops() * steps / (ftot * 1e-3) / 1e12, 2),
-                     "tflops_bwd": round(w.bwd_flops() * steps / ((tot - ftot) * 1e-3) / 1e12, 2)
-                     if tot > ftot else None,
-                     "ms_fwd_bwd": round(tot / steps, 3), "ms_fwd": round(ftot / steps, 3),
-                     "frac_of_bf16_peak": round(fl * steps / (tot * 1e-3) / 1e12 / peak, 4)}
+                     "steps_fwd_bwd": n_fb, "steps_fwd": n_f,
+                     "tflops_fwd_bwd": round(tf_fb, 2), "tflops_fwd": round(tf_f, 2),
+                     "tflops_bwd": round(tf_b, 2) if tf_b else None,
+                     "ms_fwd_bwd": round(ms_fb, 3), "ms_fwd": round(ms_f, 3),
+                     "frac_of_bf16_peak": round(tf_fb / peak, 4),
+                     "roofline": roofline_obj(tf_fb, peak, "TFLOP/s", src),
+                     "roofline_fwd": roofline_obj(tf_f, peak, "TFLOP/s", src),
+                     "roofline_bwd": roofline_obj(tf_b, peak, "TFLOP/s", src) if tf_b else None,
+                     "clocks": clk, "clocks_fwd": fclk}
         del q, k, v, do, o, dq, dk, dv, ws
     # the headline kernel at a long sequence (same kernel, B=1 H=16 N=32768 causal d=128):
     # context for the per-tile costs that weigh more at N=4096
@@ -343,13 +432,13 @@ def run_extras(fa, dev, stream, steps, peak, hbm_peak):
     o = torch.empty_like(q)
     lse = torch.empty((B_, H_, N_), dtype=torch.float32, device=dev)
     fl = 4.0 * B_ * H_ * N_ * N_ * d_ / 2
-    n_ = max(3, steps // 2)
-    tot, _ = time_steps(lambda: fa.fa_fwd(q, k, v, o, lse, causal=True, stream=stream), n_, 2,
-                        stream)
+    tot, _, n_, clk = timed_region(lambda: fa.fa_fwd(q, k, v, o, lse, causal=True, stream=stream),
+                                   steps, 2, stream, gpu)
+    tf = fl * n_ / (tot * 1e-3) / 1e12
     out["fwd_d128_long"] = {"workload": "bf16 causal forward B=1 H=16 N=32768 d=128 (N(0,1))",
-                            "tflops_fwd": round(fl * n_ / (tot * 1e-3) / 1e12, 2),
-                            "ms_fwd": round(tot / n_, 3),
-                            "frac_of_bf16_peak": round(fl * n_ / (tot * 1e-3) / 1e12 / peak, 4)}
+                            "steps": n_, "tflops_fwd": round(tf, 2), "ms_fwd": round(tot / n_, 3),
+                            "frac_of_bf16_peak": round(tf / peak, 4),
+                            "roofline": roofline_obj(tf, peak, "TFLOP/s", src), "clocks": clk}
     del q, k, v, o, lse
     # decoding: one query per sequence against a 32k KV cache, 32 query heads on 8 K/V
     # heads; memory-bound, so reported against the measured HBM bandwidth
@@ -364,9 +453,12 @@ def run_extras(fa, dev, stream, steps, peak, hbm_peak):
                      dtype=torch.uint8, device=dev)
     # the K/V cache (1.07 GB) is far larger than L2, so every launch reads it from HBM;
     # decoding steps follow one another, so the calls are timed back to back
-    calls = 50
+    calls = 200
+    clk = ClockSampler(gpu)
+    clk.start()
     tot = time_back_to_back(lambda: fa.fa_decode(q, k, v, o, lse, ws, causal=dw.causal,
                                                  stream=stream), calls, 3, stream)
+    c = clk.stop()
     gbs = dw.bytes() * calls / (tot * 1e-3) / 1e9
     out["decode_d128"] = {"workload": f"decode B={dw.B} Hq={dw.Hq} Hkv={dw.Hkv} Nq={dw.Nq} "
                                       f"Nk={dw.Nk} d={dw.d} causal",
@@ -375,8 +467,13 @@ def run_extras(fa, dev, stream, steps, peak, hbm_peak):
                           "achieved_gbs": round(gbs, 1),
                           "hbm_peak_gbs": hbm_peak,
                           "frac_of_hbm": round(gbs / hbm_peak, 4),
-                          "tflops": round(dw.flops() * calls / (tot * 1e-3) / 1e12, 2)}
+                          "tflops": round(dw.flops() * calls / (tot * 1e-3) / 1e12, 2),
+                          "roofline": roofline_obj(gbs, hbm_peak, "GB/s",
+                                                   "measured HBM copy bandwidth", bound="hbm"),
+                          "clocks": c}
     del q, k, v, o, lse, ws
+    fp8_peak = measure_fp8_peak(dev, gpu)
+    out["fp8_matmul_peak"] = fp8_peak
     w = workloads.WORKLOADS["fp8_d128"]
     gen.manual_seed(w.seed)
     shp = (w.B, w.H, w.N, w.d)
@@ -392,12 +489,18 @@ def run_extras(fa, dev, stream, steps, peak, hbm_peak):
     lse = torch.empty(shp[:3], dtype=torch.float32, device=dev)
     f8 = lambda: fa.fa_fwd_fp8(t8["q"], t8["k"], t8["v"], sc["q"], sc["k"], sc["v"], o, lse,
                                scale=w.sm_scale, causal=True, stream=stream)
-    tot, _ = time_steps(f8, steps, 2, stream)
+    tot, _, n_, clk = timed_region(f8, steps, 2, stream, gpu)
+    tf = w.fwd_flops() * n_ / (tot * 1e-3) / 1e12
+    if "tflops" in fp8_peak:
+        f8roof = roofline_obj(tf, fp8_peak["tflops"], "TFLOP/s",
+                              "measured e4m3 dense matmul (torch._scaled_mm, burst)")
+    else:
+        f8roof = roofline_obj(tf, 2 * peak, "TFLOP/s",
+                              "2x the measured bf16 matmul peak (nominal FP8/bf16 ratio)")
     out["fp8_d128"] = {"workload": "FP8 e4m3 causal forward B=1 H=32 N=32768 d=128",
-                       "tflops_fwd": round(w.fwd_flops() * steps / (tot * 1e-3) / 1e12, 2),
-                       "ms_fwd": round(tot / steps, 3),
-                       "frac_of_fp8_nominal_2x_bf16_peak":
-                           round(w.fwd_flops() * steps / (tot * 1e-3) / 1e12 / (2 * peak), 4)}
+                       "steps": n_, "tflops_fwd": round(tf, 2), "ms_fwd": round(tot / n_, 3),
+                       "frac_of_fp8_nominal_2x_bf16_peak": round(tf / (2 * peak), 4),
+                       "roofline": f8roof, "clocks": clk}
     # FP8 backward on the same inputs: dequantisation passes + the bf16 backward
     gen.manual_seed(w.seed + 1)
     do = torch.randn(shp, generator=gen, device=dev).to(torch.bfloat16)
@@ -406,13 +509,42 @@ def run_extras(fa, dev, stream, steps, peak, hbm_peak):
     f8()
     b8 = lambda: fa.fa_bwd_fp8(t8["q"], t8["k"], t8["v"], sc["q"], sc["k"], sc["v"], o, do, lse,
                                dq, dk, dv, ws, scale=w.sm_scale, causal=True, stream=stream)
-    bsteps = max(3, steps // 3)
-    btot, _ = time_steps(b8, bsteps, 1, stream)
+    btot, _, bn, bclk = timed_region(b8, steps, 1, stream, gpu)
+    tb = w.bwd_flops() * bn / (btot * 1e-3) / 1e12
     out["fp8_d128"].update({
-        "tflops_bwd": round(w.bwd_flops() * bsteps / (btot * 1e-3) / 1e12, 2),
-        "ms_bwd": round(btot / bsteps, 3),
+        "steps_bwd": bn, "tflops_bwd": round(tb, 2), "ms_bwd": round(btot / bn, 3),
+        "roofline_bwd": roofline_obj(tb, peak, "TFLOP/s", src + "; the backward runs in bf16"),
+        "clocks_bwd": bclk,
         "bwd_note": "gradients for the dequantised inputs: e4m3 -> bf16 pass, then the bf16 "
                     "backward (metric FLOPs 2.5x the forward's)"})
+    return out
+
+
+def cpu_sdpa_figure():
+    """The pages' CPU measurement repeated on this host: torch scaled_dot_product_attention
+    in fp32 on the CPU, MATH and FLASH backends, B=1 H=8 d=64 causal, N = 1024/2048/4096
+    (the [issoh] CPU table prints 66.3 ms MATH and 14.0 ms FLASH at N=1024 on an
+    8-thread i9-9880H).  Median of 5 calls after one warm-up; context, not a target."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    out = {"threads": torch.get_num_threads(), "cores": _cores(),
+           "workload": "fp32 CPU SDPA B=1 H=8 d=64 causal", "ms": {}}
+    gen = torch.Generator().manual_seed(1001)
+    for n in (1024, 2048, 4096):
+        q, k, v = (torch.randn((1, 8, n, 64), generator=gen) for _ in range(3))
+        row = {}
+        for name, be in (("math", SDPBackend.MATH), ("flash", SDPBackend.FLASH_ATTENTION)):
+            try:
+                with sdpa_kernel(be):
+                    torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+                    ts = []
+                    for _ in range(5):
+                        t0 = time.perf_counter()
+                        torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+                        ts.append((time.perf_counter() - t0) * 1e3)
+                row[name] = round(statistics.median(ts), 2)
+            except RuntimeError as e:
+                row[name] = f"unavailable: {str(e).splitlines()[0][:120]}"
+        out["ms"][str(n)] = row
     return out
 
 
@@ -485,7 +617,9 @@ def run_reference(args):
 
 def run_profile_driver(name, launches):
     """Launch one workload's kernels a few times and exit: the target for ncu captures
-    (`ncu -k regex:... -s <skip> -c <n> python bench.py --profile <name>`)."""
+    (`ncu --clock-control none -k regex:... -s <skip> -c <n> python bench.py --profile
+    <name>`).  Always pass --clock-control none (ncu otherwise locks the GPU clocks),
+    and keep a capture beyond gpu__time_duration.sum to one kernel and a few launches."""
     import exact_attention_132_b200 as fa
     w = workloads.WORKLOADS[name]
     dev = torch.device("cuda", 0)

@@ -17,7 +17,8 @@ import torch
 
 __all__ = [
     "FAError", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_size", "fa_last_error_string",
-    "fa_get_device_status", "fa_debug_wait_timeout_selftest", "fa_version", "fa_fwd_kernel_name",
+    "fa_get_device_status", "fa_debug_wait_timeout_selftest", "fa_debug_exp2", "fa_version",
+    "fa_fwd_kernel_name",
     "fa_decode", "fa_decode_workspace_size", "fa_fwd_gqa", "fa_bwd_gqa", "attention_forward",
     "attention_decode", "attention_forward_gqa", "attention_backward_gqa",
     "attention_forward_fp8", "attention_backward", "LIB_PATH", "lib",
@@ -53,6 +54,8 @@ def _load() -> ctypes.CDLL:
     L.fa_last_error_string.restype = ctypes.c_char_p
     L.fa_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     L.fa_debug_wait_timeout_selftest.argtypes = [i, vp]
+    L.fa_debug_exp2.argtypes = [vp, vp, vp, vp, i, vp]
+    L.fa_debug_exp2.restype = ctypes.c_int
     L.fa_version.argtypes = []
     L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     L.fa_fwd_gqa.restype = ctypes.c_int
@@ -200,6 +203,15 @@ def fa_get_device_status(stream=None) -> int:
 
 def fa_debug_wait_timeout_selftest(timeout_us: int, stream=None) -> None:
     _check(lib.fa_debug_wait_timeout_selftest(int(timeout_us), _stream(stream)))
+
+
+def fa_debug_exp2(x: torch.Tensor, stream=None):
+    """(software 2^x, special-function-unit ex2, exp2f) of the fp32 CUDA tensor x."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    outs = tuple(torch.empty_like(x) for _ in range(3))
+    _check(lib.fa_debug_exp2(_ptr(x), *(_ptr(t) for t in outs), x.numel(), _stream(stream)))
+    return outs
 
 
 def fa_version() -> int:

@@ -94,7 +94,10 @@ fa_status device_info(DeviceInfo** out) {
 
 // The scheduler counter pair of `stream`.  Streams get slots in order of first use;
 // beyond kSchedSlots distinct streams the slots are reused round-robin, so at most
-// kSchedSlots streams may run forwards on one device at the same time.
+// kSchedSlots streams may run forwards on one device at the same time.  Slots are
+// keyed by the stream handle: a stream destroyed while its forwards are still queued
+// and a new stream that receives the same handle would share one counter pair, so a
+// stream's forwards must finish before the stream is destroyed (stated in fa.h).
 int* sched_counter(DeviceInfo* d, cudaStream_t stream) {
   std::lock_guard<std::mutex> lock(d->sched_mu);
   const int n = d->sched_used < kSchedSlots ? d->sched_used : kSchedSlots;
@@ -495,6 +498,27 @@ __global__ void wait_selftest_kernel(unsigned* status, unsigned long long timeou
   // Nothing ever arrives on `bar`: the wait has to run out and report.
   mbar_wait(smem_u32(&bar), 0, wc, kSiteSelfTest);
   __syncthreads();
+}
+
+// Evaluates the kernels' exponential helpers on n values: the software exp2 of the
+// FMA pipe (ex2_poly_pair, two values per call), the special-function-unit ex2 and
+// CUDA's exp2f, for the accuracy test of the software exp2.
+__global__ void exp2_probe_kernel(const float* x, float* y_poly, float* y_sfu, float* y_exp2f,
+                                  int n) {
+  const long long i = 2ll * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const bool two = i + 1 < n;
+  const float a = x[i], b = two ? x[i + 1] : 0.f;
+  float pa, pb;
+  f2_unpack(ex2_poly_pair(f2_pack(a, b)), pa, pb);
+  y_poly[i] = pa;
+  y_sfu[i] = ex2(a);
+  y_exp2f[i] = exp2f(a);
+  if (two) {
+    y_poly[i + 1] = pb;
+    y_sfu[i + 1] = ex2(b);
+    y_exp2f[i + 1] = exp2f(b);
+  }
 }
 
 size_t workspace_bytes(int B, int H, int N) {
@@ -1032,6 +1056,21 @@ fa_status fa_debug_wait_timeout_selftest(int timeout_us, void* stream) {
       di->status, static_cast<unsigned long long>(timeout_us) * 1000ull);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return FA_OK;
+}
+
+fa_status fa_debug_exp2(const float* x, float* y_poly, float* y_sfu, float* y_exp2f, int n,
+                        void* stream) {
+  if (n < 0) return fail(FA_ERR_INVALID_ARG, "n = %d is negative", n);
+  if (n == 0) return FA_OK;
+  if (!x || !y_poly || !y_sfu || !y_exp2f) return fail(FA_ERR_INVALID_ARG, "null pointer");
+  const int threads = 256;
+  const long long pairs = (static_cast<long long>(n) + 1) / 2;
+  const unsigned blocks = static_cast<unsigned>((pairs + threads - 1) / threads);
+  exp2_probe_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_sfu,
+                                                                                 y_exp2f, n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "exp2 probe launch");
   return FA_OK;
 }
 

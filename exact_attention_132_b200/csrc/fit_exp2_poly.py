@@ -11,7 +11,7 @@ float32-Horner evaluation against float64 2^f.
 
     python exact_attention_132_b200/csrc/fit_exp2_poly.py [--degree 3]
 
-The printed coefficients are pasted into fa_fwd.cuh (kExp2Poly).
+The printed coefficients are the constants kC0..kC3 of ex2_poly_pair in sm100_ptx.cuh.
 """
 from __future__ import annotations
 

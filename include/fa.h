@@ -22,14 +22,17 @@
  *  Pointers  device pointers (cudaMalloc / torch CUDA memory) on the current
  *            device, 16-byte aligned.  The caller owns every buffer; the
  *            library allocates and frees no device memory on any call.
- *  Sizes     B, H, N >= 0; d in {64, 128, 256} (bf16) or {128} (FP8).  N need
+ *  Sizes     B, H, N >= 0; d in {64, 96, 128, 192, 256} (bf16 and FP8).  N need
  *            not be a multiple of 128.  A call with B*H*N == 0 returns FA_OK
  *            and launches nothing (pointers may then be NULL).
  *  causal    0 = every key visible; 1 = key j visible to query i iff j <= i
  *            (lower triangular, top-left aligned; N_q == N_k).
  *  scale     multiplier of Q K^T, finite and > 0 (SDPA's default is 1/sqrt(d)).
  *  Streams   every call is asynchronous on `stream` (a cudaStream_t, 0 = the
- *            legacy default stream) and never synchronises the host.
+ *            legacy default stream) and never synchronises the host.  The
+ *            forwards keep a small work counter per stream handle: let a
+ *            stream's forwards finish before destroying the stream, since a
+ *            stream created afterwards may receive the same handle.
  *  Errors    argument errors return at once, before any CUDA call, and launch
  *            nothing.  There is no fallback path: an unsupported request fails
  *            (issoh.co.jp page, section CPUのPyTorch SDPA…: a forced fused path
@@ -258,7 +261,7 @@ size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
  *   k, v       bf16 [B, Hkv, Nk, d]                    (device, read)
  *   o          bf16 [B, Hq, Nq, d]                     (device, written)
  *   lse        fp32 [B, Hq, Nq] natural-log logsumexp  (device, written; may be NULL)
- *   d in {64, 128, 256}; Hq % Hkv == 0; (Hq / Hkv) * Nq <= 128; 1 <= Nq; 1 <= Nk;
+ *   d in {64, 96, 128, 192, 256}; Hq % Hkv == 0; (Hq / Hkv) * Nq <= 128; 1 <= Nq; 1 <= Nk;
  *   causal requires Nq <= Nk.
  *   workspace  >= fa_decode_workspace_size() bytes of device memory, 16-byte aligned,
  *              owned by the caller, contents ignored and overwritten.
@@ -288,6 +291,20 @@ fa_status fa_get_device_status(void* stream, int* code);
  * return; the context stays usable.  Used by the tests of the fault path.
  */
 fa_status fa_debug_wait_timeout_selftest(int timeout_us, void* stream);
+
+/*
+ * fa_debug_exp2 — evaluates, for the n fp32 values x[0..n-1], the exponential
+ * helpers the kernels use: y_poly = the software 2^x on the FMA pipe (Cody-Waite
+ * reduction and a degree-3 minimax polynomial; FA4's partial software exponential,
+ * "FlashAttentionとは？…" (issoh.co.jp), section FA4のB200で1613TFLOPs…), y_sfu =
+ * the special-function unit's ex2.approx.ftz, y_exp2f = CUDA's exp2f.  All four
+ * are fp32 device arrays of n elements owned by the caller.  The software form is
+ * specified for x <= 127 with relative error <= 7.5e-5 on (-126, 127]; inputs at or
+ * below -126 give a value in [0, 2^-126].  n < 0 or a null pointer with n > 0:
+ * FA_ERR_INVALID_ARG.  Used by the accuracy test of the software exponential.
+ */
+fa_status fa_debug_exp2(const float* x, float* y_poly, float* y_sfu, float* y_exp2f, int n,
+                        void* stream);
 
 /* fa_version — library version, major*10000 + minor*100 + patch. */
 int fa_version(void);

@@ -32,6 +32,40 @@ def _close(a, b, tol):
     return a.shape == b.shape and bool(np.all(np.abs(a - b) <= tol))
 
 
+# --------------------------------------------------------------------------- softmax weights
+def check_softmax_probs_brute(probs, N=9, d=4) -> bool:
+    """The probability matrix P equals the attention weights of the pure-Python brute
+    force: with V = the N x N identity, O = P V = P row by row.  Q and K are drawn
+    independently, so Q K^T is not symmetric and a transposed score matrix fails."""
+    rng = _rng(21)
+    q, k = rng.standard_normal((2, N, d)) * 1.5
+    eye = np.eye(N).tolist()
+    for causal in (False, True):
+        want, _ = brute_fwd(q.tolist(), k.tolist(), eye, 0.6, causal)
+        got = probs(q[None, None], k[None, None], 0.6, causal)[0, 0]
+        if not _close(got, want, 1e-13):
+            return False
+        if causal and np.any(np.triu(got, 1) != 0):
+            return False
+    return True
+
+
+def check_softmax_rows_sum_to_one(probs, N=64, d=16) -> bool:
+    """Rows of P are non-negative and sum to one; causal P vanishes above the diagonal."""
+    rng = _rng(3)
+    q, k = (rng.standard_normal((1, 2, N, d)) * 3 for _ in range(2))
+    for causal in (False, True):
+        P = probs(q, k, 0.25, causal)
+        if not (np.all(P >= 0) and np.abs(P.sum(-1) - 1).max() < 1e-14):
+            return False
+        if causal and np.any(P[..., np.triu_indices(N, 1)[0], np.triu_indices(N, 1)[1]] != 0):
+            return False
+    return True
+
+
+PROBS_CHECKS = [check_softmax_probs_brute, check_softmax_rows_sum_to_one]
+
+
 # --------------------------------------------------------------------------- forward checks
 def check_golden_tiny_fwd(fwd) -> bool:
     """Hand-derived N=2, d=1 example (tests/golden/tiny_closed_form.json)."""

@@ -182,3 +182,11 @@ def test_noalloc_backward_argument_errors_return_before_any_cuda_call():
     assert "dq" in fa.fa_last_error_string()
     # empty problems launch nothing and touch no pointer
     assert call(B=0, ps=[None] * 9) == fa.FA_OK
+
+
+def test_exp2_probe_argument_errors_return_before_any_cuda_call():
+    P = ctypes.c_void_p(256)
+    assert fa.lib.fa_debug_exp2(P, P, P, P, -1, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.lib.fa_debug_exp2(None, P, P, P, 8, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.lib.fa_debug_exp2(P, P, None, P, 8, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.lib.fa_debug_exp2(None, None, None, None, 0, None) == fa.FA_OK

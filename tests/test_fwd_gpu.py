@@ -49,26 +49,28 @@ def test_fwd_small_workload_full(fa):
     print("fwd_small", err)
 
 
-def test_fwd_outlier_workload_full_size_sampled(fa):
+def test_fwd_outlier_workload_full_size_every_element(fa):
     """B=4 H=16 N=4096 d=128 causal with 1% K outlier rows, run at full size in the
-    benchmark's launch configuration; sampled rows are checked one by one against the
-    oracle (each sampled row still sees all of its keys)."""
+    benchmark's launch configuration (persistent grid, dynamic item draw): every row of
+    every head is checked against the oracle, so every work item the scheduler hands out
+    is covered."""
     w = workloads.WORKLOADS["fwd_d128"]
     q, k, v = workloads.make_bf16_inputs(w)
     o, lse = fa.attention_forward(q.cuda(), k.cuda(), v.cuda(), causal=True, scale=w.sm_scale)
-    picks = parity.sample_rows(w.B, w.H, w.N, n_heads=6, n_rows=40, seed=2)
-    o_ref, lse_ref = oracle.attention_fwd_rows(q, k, v, w.sm_scale, True, picks)
+    torch.cuda.synchronize()
     og, lg = o.cpu(), lse.cpu()
-    got_o = np.stack([parity.to64(og[b, h, i]) for b, h, i in picks])
-    got_l = np.array([float(lg[b, h, i]) for b, h, i in picks])
-    err = parity.assert_fwd_ok(got_o, got_l, o_ref, lse_ref, tag=w.name)
-    print("fwd_d128 sampled", err)
-    # whole-output properties that hold at any size
-    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    worst = {"o_max_abs": 0.0, "o_mean_abs": 0.0, "lse_max_rel": 0.0}
+    for b in range(w.B):
+        # one batch entry (16 heads) at a time keeps the fp64 copies small
+        o_ref, lse_ref = oracle.attention_fwd(q[b:b + 1], k[b:b + 1], v[b:b + 1], w.sm_scale, True)
+        err = parity.assert_fwd_ok(og[b:b + 1], lg[b:b + 1], o_ref, lse_ref, tag=(w.name, b))
+        for key in worst:
+            worst[key] = max(worst[key], err[key])
+    print("fwd_d128 every element", worst)
     # causal row 0 of every head is V_0 exactly (a single visible key) and LSE_0 = scale q0.k0
-    assert torch.equal(o[:, :, 0].cpu(), v[:, :, 0])
+    assert torch.equal(og[:, :, 0], v[:, :, 0])
     ref_l0 = (q[:, :, 0].double() * k[:, :, 0].double()).sum(-1) * w.sm_scale
-    assert (lse[:, :, 0].cpu().double() - ref_l0).abs().max() < 1e-3 * max(1.0, ref_l0.abs().max())
+    assert (lg[:, :, 0].double() - ref_l0).abs().max() < 1e-3 * max(1.0, ref_l0.abs().max())
 
 
 def test_fwd_is_deterministic(fa):

@@ -208,3 +208,35 @@ def test_gqa_backward_mutant_is_caught(name):
     kw = MUTANTS_GQA_BWD[name]
     f = lambda q, k, v, do, s, c: _gqa_bwd_generic(q, k, v, do, s, c, **kw)
     assert not all(chk(f) for chk in oc.GQA_BWD_CHECKS), f"mutant {name} passed every check"
+
+
+def _probs_generic(q, k, scale, causal, *, transpose=False, axis=-1, use_scale=True):
+    q, k = (np.asarray(x, dtype=np.float64) for x in (q, k))
+    s = (k @ np.swapaxes(q, -1, -2)) if transpose else (q @ np.swapaxes(k, -1, -2))
+    if use_scale:
+        s = s * scale
+    if causal:
+        N = s.shape[-1]
+        s = np.where(np.triu(np.ones((N, N), bool), 1), -np.inf, s)
+    e = np.exp(s - s.max(axis=axis, keepdims=True))
+    return e / e.sum(axis=axis, keepdims=True)
+
+
+def test_unmutated_probs_pass():
+    for chk in oc.PROBS_CHECKS:
+        assert chk(lambda q, k, s, c: _probs_generic(q, k, s, c)), chk.__name__
+
+
+@pytest.mark.parametrize("kw", [dict(transpose=True), dict(axis=-2), dict(use_scale=False)],
+                         ids=["transposed_scores", "wrong_axis", "dropped_scale"])
+def test_probs_mutant_is_caught(kw):
+    f = lambda q, k, s, c: _probs_generic(q, k, s, c, **kw)
+    failures = []
+    for chk in oc.PROBS_CHECKS:
+        try:
+            ok = chk(f)
+        except Exception:
+            ok = False
+        if not ok:
+            failures.append(chk.__name__)
+    assert failures, f"softmax_probs mutant {kw} passed every check"

@@ -25,16 +25,10 @@ def test_oracle_matches_pages_fp32_magnitude():
     assert oc.check_fp32_sdpa_magnitude(oracle.attention_fwd)
 
 
-def test_softmax_rows_normalised():
-    """Rows of P sum to one and P vanishes above the diagonal when causal."""
-    rng = np.random.default_rng(3)
-    q, k = (rng.standard_normal((1, 2, 64, 16)) * 3 for _ in range(2))
-    for causal in (False, True):
-        P = oracle.softmax_probs(q, k, 0.25, causal)
-        assert np.all(P >= 0)
-        assert np.abs(P.sum(-1) - 1).max() < 1e-14
-        if causal:
-            assert np.all(P[..., np.triu_indices(64, 1)[0], np.triu_indices(64, 1)[1]] == 0)
+@pytest.mark.parametrize("check", oc.PROBS_CHECKS, ids=lambda f: f.__name__)
+def test_softmax_probs_pins(check):
+    """P from the two-pass definition: rows sum to one, and P is the brute force's weights."""
+    assert check(oracle.softmax_probs)
 
 
 @pytest.mark.parametrize("causal", [False, True])
