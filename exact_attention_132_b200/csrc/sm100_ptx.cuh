@@ -422,7 +422,11 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 // f in [-1/2, 1/2]; 2^f by a degree-3 polynomial with minimax relative error 7.5e-5
 // (coefficients from csrc/fit_exp2_poly.py); 2^n by adding n << 23 to the
 // exponent field.  x is clamped at -126 (the result there, about 1.2e-38, stands in
-// for anything smaller), so the exponent field never underflows; valid for x <= 127.
+// for anything smaller); valid for x <= 127.  Relative error <= 7.5e-5 on
+// (-125.99, 127]; on [-126, -125.99] the polynomial can fall just below one while
+// 2^n = 2^-126, the exponent field then reaches zero and the subnormal encoding
+// drops the implicit leading bit: error <= 1.5e-4 there (values near 1e-38, which
+// no softmax sum can see).
 // Callers keep -inf away from it: the forward uses it only on tiles with no masked
 // scores, the backward replaces masked entries after the call.
 __device__ __forceinline__ uint64_t ex2_poly_pair(uint64_t x2) {

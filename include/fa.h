@@ -299,8 +299,9 @@ fa_status fa_debug_wait_timeout_selftest(int timeout_us, void* stream);
  * "FlashAttentionとは？…" (issoh.co.jp), section FA4のB200で1613TFLOPs…), y_sfu =
  * the special-function unit's ex2.approx.ftz, y_exp2f = CUDA's exp2f.  All four
  * are fp32 device arrays of n elements owned by the caller.  The software form is
- * specified for x <= 127 with relative error <= 7.5e-5 on (-126, 127]; inputs at or
- * below -126 give a value in [0, 2^-126].  n < 0 or a null pointer with n > 0:
+ * specified for x <= 127 with relative error <= 7.5e-5 on (-125.99, 127] and
+ * <= 1.5e-4 on [-126, -125.99] (a subnormal encoding there); inputs at or below
+ * -126 give a value in [0, 2^-126].  n < 0 or a null pointer with n > 0:
  * FA_ERR_INVALID_ARG.  Used by the accuracy test of the software exponential.
  */
 fa_status fa_debug_exp2(const float* x, float* y_poly, float* y_sfu, float* y_exp2f, int n,
