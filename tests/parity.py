@@ -1,9 +1,19 @@
 """Shared comparison helpers and tolerances for the GPU-vs-oracle parity tests.
 
 Tolerances (stated once, used everywhere):
-  bf16 forward : O max |err| <= 1e-2, O mean |err| <= 1e-3, LSE max relative err <= 1e-3
+  bf16 forward : O max |err| <= 1e-2 beyond the rounding of the output to bf16 (see
+                 below), O mean |err| <= 1e-3, LSE max relative err <= 1e-3
   bf16 backward: relative Frobenius error <= 2e-2 for each of dQ, dK, dV
-  FP8 forward  : O max |err| <= 6e-2 (against the oracle on the dequantised inputs)
+  FP8 forward  : O max |err| <= 6e-2 beyond the output rounding (against the oracle on
+                 the dequantised inputs)
+
+Output rounding.  O is returned in bf16 (the workloads fix it: "outputs O (bf16)").
+Near |O| >= 4 the bf16 grid is 2^-5 apart, so even the exact result rounded to bf16
+misses it by up to 2^-6 = 0.0156 > 1e-2: no bf16 output could meet a plain 1e-2 bound
+there.  The max-abs bounds are therefore read as bounds on the kernel's arithmetic
+error beyond that last rounding: per element |O - O*| <= tol + ulp_bf16(O*) / 2.  The
+mean bound stays plain.  (Found by the every-element check of the B4 H16 N4096 d128
+workload: max |err| 0.0188 at |O*| in [4, 8), where half an ulp is 0.0156.)
 """
 from __future__ import annotations
 
@@ -23,11 +33,22 @@ def to64(t) -> np.ndarray:
     return np.asarray(t, dtype=np.float64)
 
 
+def half_ulp_bf16(x) -> np.ndarray:
+    """Half the spacing of the bf16 grid at |x| (8 significant bits): 2^(e - 8) for
+    2^e <= |x| < 2^(e+1); 0 at x = 0."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(e - 8), 0.0)
+
+
 def fwd_errors(o, lse, o_ref, lse_ref) -> dict:
     o, lse = to64(o), to64(lse)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
     e = np.abs(o - o_ref)
     return {
         "o_max_abs": float(e.max()) if e.size else 0.0,
+        # the error beyond the output's own rounding to bf16
+        "o_max_beyond_rounding": float((e - half_ulp_bf16(o_ref)).max()) if e.size else 0.0,
         "o_mean_abs": float(e.mean()) if e.size else 0.0,
         "lse_max_rel": float((np.abs(lse - lse_ref) / np.maximum(np.abs(lse_ref), 1e-30)).max())
         if lse.size else 0.0,
@@ -35,9 +56,14 @@ def fwd_errors(o, lse, o_ref, lse_ref) -> dict:
     }
 
 
+def o_ok(err: dict, tol: float) -> bool:
+    """The per-element max-abs bound beyond the output rounding."""
+    return err["o_max_beyond_rounding"] <= tol
+
+
 def assert_fwd_ok(o, lse, o_ref, lse_ref, tag=""):
     err = fwd_errors(o, lse, o_ref, lse_ref)
-    assert err["o_max_abs"] <= O_MAX_ABS, (tag, err)
+    assert o_ok(err, O_MAX_ABS), (tag, err)
     assert err["o_mean_abs"] <= O_MEAN_ABS, (tag, err)
     # LSE relative error: the pages' reading is "relative"; near LSE = 0 (causal row 0
     # with q0.k0 ~ 0) a relative bound is meaningless, so small |LSE| use an absolute 1e-3.
