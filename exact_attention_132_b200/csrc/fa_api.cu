@@ -264,19 +264,17 @@ fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p
   return FA_OK;
 }
 
-// Tuning knobs (compile-time): software-exp2 share, pipeline depth, kernel family.
-// software-exp2 share (quarters of the exponentials) per problem class, measured: the
-// two-tile kernel wants 1 at d = 64 and FP8 (2 and 3 were slower) and none at bf16
-// d = 128 (its per-step path is issue-bound there, not bound by the special-function
-// unit); the d = 256 kernel (tensor-core bound) none
+// Tuning knobs (compile-time): software-exp2 share, pipeline depth, softmax layout.
+// Software-exp2 share of the two-tile kernel, in pairs of every 16 exponential pairs,
+// per problem class; the one-tile d = 256 kernel counts quarters.
 #ifndef FA_FWD_EMU
 #define FA_FWD_EMU 0
 #endif
 #ifndef FA_FWD_D64_EMU
-#define FA_FWD_D64_EMU 1
+#define FA_FWD_D64_EMU 4
 #endif
 #ifndef FA_FWD_F8_EMU
-#define FA_FWD_F8_EMU 1
+#define FA_FWD_F8_EMU 4
 #endif
 #ifndef FA_FWD_D256_EMU
 #define FA_FWD_D256_EMU 0
@@ -299,57 +297,35 @@ fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p
 // (measured: +6.7 % on N(0,1) inputs at N = 32768, +1 % at d = 64, neutral on the
 // outlier-key headline workload whose max jumps exceed the threshold)
 #ifndef FA_FWD_TAU
-#define FA_FWD_TAU 8
+#define FA_FWD_TAU 4
 #endif
-#ifndef FA_FWD_PP_COMP
-#define FA_FWD_PP_COMP 1
+#ifndef FA_FWD_PP_NORM
+#define FA_FWD_PP_NORM 1
 #endif
-#ifndef FA_FWD_EXPH
-#define FA_FWD_EXPH 0
-#endif
-// Kernel family per problem class (measured fastest on the causal N = 4096 workloads):
-// 0 = one query tile per CTA (fa_fwd.cuh), 1 = two query tiles (fa_fwd_pp.cuh).
-#ifndef FA_FWD_D64_KIND
-#define FA_FWD_D64_KIND 1
-#endif
-#ifndef FA_FWD_D128_KIND
-#define FA_FWD_D128_KIND 1
-#endif
-#ifndef FA_FWD_F8_KIND
-#define FA_FWD_F8_KIND 1
-#endif
-
-template <int KIND, int D, bool FP8, int EMU>
+template <int D, bool FP8, int EMU>
 struct FwdPick {
   // stage depths: deep rings where shared memory allows, 2 + 2 for bf16 d = 128
   static constexpr bool kWide = (D == 128 && !FP8);
   static constexpr int KST = kWide ? FA_FWD_D128_KST : FA_FWD_NARROW_ST;
   static constexpr int VST = kWide ? FA_FWD_D128_VST : FA_FWD_NARROW_ST;
-  using Cfg = std::conditional_t<
-      KIND == 0, FwdCfg<D, 128, kWide ? 3 : 4, kWide ? 2 : 4, FP8, EMU>,
-      PPCfg<D, KST, VST, FP8, EMU, FA_FWD_TAU, FA_FWD_EXPH, FA_FWD_PP_COMP != 0>>;
-  static_assert(KIND == 0 || KIND == 1, "kernel family 0 or 1");
+  using Cfg = PPCfg<D, KST, VST, FP8, EMU, FA_FWD_TAU, FA_FWD_PP_NORM>;
   static const char* name() {
     static const std::string n = [] {
-      static const char* fam[] = {"fa_fwd_kernel<FwdCfg", "fa_fwd_pp_kernel<PPCfg"};
       char buf[128];
-      std::snprintf(buf, sizeof buf, "%s<%d,KST%d,VST%d,%s>>", fam[KIND], D, Cfg::KST, Cfg::VST,
-                    FP8 ? "e4m3" : "bf16");
+      std::snprintf(buf, sizeof buf, "fa_fwd_pp_kernel<PPCfg<%d,KST%d,VST%d,%s>>", D, Cfg::KST,
+                    Cfg::VST, FP8 ? "e4m3" : "bf16");
       return std::string(buf);
     }();
     return n.c_str();
   }
   static fa_status launch(const void* q, const void* k, const void* v, FwdParams p,
                           cudaStream_t st) {
-    if constexpr (KIND == 0)
-      return launch_fwd<Cfg>(q, k, v, p, st);
-    else
-      return launch_fwd_pp<Cfg>(q, k, v, p, st);
+    return launch_fwd_pp<Cfg>(q, k, v, p, st);
   }
 };
-using FwdD64 = FwdPick<FA_FWD_D64_KIND, 64, false, FA_FWD_D64_EMU>;
-using FwdD128 = FwdPick<FA_FWD_D128_KIND, 128, false, FA_FWD_EMU>;
-using FwdF8D128 = FwdPick<FA_FWD_F8_KIND, 128, true, FA_FWD_F8_EMU>;
+using FwdD64 = FwdPick<64, false, FA_FWD_D64_EMU>;
+using FwdD128 = FwdPick<128, false, FA_FWD_EMU>;
+using FwdF8D128 = FwdPick<128, true, FA_FWD_F8_EMU>;
 using FwdD256 = FwdCfg<256, 64, 3, 2, false, FA_FWD_D256_EMU, FA_FWD_D256_TAU>;
 using FwdF8D256 = FwdCfg<256, 128, 3, 2, true, FA_FWD_F8_EMU>;
 

@@ -3,18 +3,19 @@
 // Same mathematics as fa_fwd.cuh (tiled S = Q K^T, exp2 online softmax with the
 // output rescaled only when a row max rises, O += P V, causal tile skip), but a
 // work item is a PAIR of 128-row query tiles of one head that share every K/V tile
-// load, and each tile has its own softmax warpgroup.  The tensor core alternates
+// load, and each tile has its own softmax warps.  The tensor core alternates
 // between the tiles:
 //
 //      ... PV_0(j-1)  S_0(j)  PV_1(j-1)  S_1(j)  PV_0(j)  S_0(j+1) ...
 //
-// so while one warpgroup turns S_t(j) into P_t(j), the tensor core works on the
+// so while one tile's warps turn S_t(j) into P_t(j), the tensor core works on the
 // other tile.  Because PV_t(j-1) is issued before S_t(j) and tcgen05 operations
 // complete in order, "S_t(j) is ready" also means "PV_t(j-1) has finished": the
-// softmax warpgroup may rescale O_t right away, with no separate wait.
+// softmax warps may rescale O_t right away, with no separate wait.
 //
 // Roles: warps 0-3 softmax for tile 0, warps 4-7 softmax for tile 1 (TMEM lane
-// quadrant = warp % 4), warp 8 TMA producer, warp 9 MMA issuer + TMEM owner.
+// quadrant = warp % 4; a thread owns one 128-key score row), warp 8 TMA producer,
+// warp 9 MMA issuer + TMEM owner.
 // Tensor memory: S_0 [0,128), S_1 [128,256), O_0 [256, 256+D), O_1 [256+D, 256+2D);
 // P_t overwrites the first columns of S_t after they are read.
 #pragma once
@@ -23,32 +24,30 @@
 
 namespace fa {
 
-template <int D_, int KST_, int VST_, bool FP8_, int EMU_ = 1, int TAU_ = 0, bool EXPH_ = false,
-          bool COMP_ = false>
+template <int D_, int KST_, int VST_, bool FP8_, int EMU_ = 0, int TAU_ = 0, int NORM_ = 0>
 struct PPCfg {
   static constexpr int D = D_;
   static constexpr int BN = 128;
   static constexpr int BM = 128;                     // rows of one query tile
   static constexpr int KST = KST_, VST = VST_;
   static constexpr bool FP8 = FP8_;
+  // Of every 16 pairs of exponentials in a score row, EMU are evaluated by the software
+  // exp2 on the FMA/ALU pipes (ex2_poly_pair) instead of the special-function unit, on
+  // tiles without masked scores.
   static constexpr int EMU = EMU_;
-  // bf16 only: the reference max used for the exponentials moves (and O is
-  // rescaled) only when a row max exceeds it by more than TAU (log2 units), so
-  // P <= 2^TAU.  With TAU > 0 the row sum l adds the bf16-ROUNDED probabilities, the
-  // very values the P V product uses, so O = sum P V / sum P is a convex combination
-  // whose weights carry no bias from rounding the largest probability; the logsumexp
-  // uses a second, unrounded sum.
+  // bf16 only: the reference max used for the exponentials moves (and O is rescaled)
+  // only when a row max exceeds it by more than TAU (log2 units), so P <= 2^TAU.
   static constexpr float TAU = FP8 ? 0.f : static_cast<float>(TAU_);
-  // bf16 only: exponentials on the special-function unit in half precision, two
-  // values per instruction (ex2.approx.f16x2).
-  static constexpr bool EXPH = EXPH_ && !FP8;
-  // TAU > 0 without the per-element rounded sum: the row sum adds the unrounded
-  // probabilities plus, per key tile, the bf16 rounding error of the tile's largest
-  // probability (the one that may exceed 1 and dominate the row).  The P V product
-  // uses every probability rounded; only the largest one's error is large enough to
-  // bias O, and it is the one the denominator takes on.  The logsumexp uses the
-  // plain unrounded sum.
-  static constexpr bool COMP = COMP_ && TAU > 0.f && !EXPH;
+  // The row sum that normalises O (bf16 with TAU > 0, where a probability can reach
+  // 2^TAU and its bf16 rounding no longer averages out):
+  //   NORM 1: the unrounded probabilities plus, per key tile, the bf16 rounding error of
+  //           the tile's largest probability;
+  //   NORM 2: the bf16-rounded probabilities themselves, the very weights of the P V
+  //           product, so O is their convex combination of V rows.
+  // The logsumexp always uses the plain unrounded sum.
+  static constexpr int NORM = (FP8 || TAU == 0.f) ? 0 : NORM_;
+  static constexpr bool COMP = NORM == 1;
+  static constexpr bool RSUM = NORM == 2;
   static constexpr int ELEM = FP8 ? 1 : 2;
   static constexpr int ROW_BYTES = D * ELEM;
   static constexpr int NBOX = ROW_BYTES / 128;
@@ -68,7 +67,8 @@ struct PPCfg {
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ITEM = SMEM_MISC + 64;    // work-item ring
   static constexpr int SMEM_ALLOC = SMEM_ITEM + kItemBytes + 1024;
-  static constexpr uint32_t ITEM_READERS = 1 + 8;     // the MMA thread and 8 softmax warps
+  static constexpr int SOFTMAX_WARPS = 8;
+  static constexpr uint32_t ITEM_READERS = 1 + SOFTMAX_WARPS;   // the MMA thread and the softmax warps
   static constexpr int TM_S = 0;                     // + t * BN
   static constexpr int TM_O = 2 * BN;                // + t * D
   static constexpr int TM_COLS = 512;
@@ -83,6 +83,7 @@ struct PPCfg {
   static_assert(REGS_TOTAL <= THREADS * 168, "register split");
   static_assert(2 * BN + 2 * D <= TM_COLS, "tensor memory budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+  static_assert(EMU >= 0 && EMU <= 16, "software exponentials per 16 pairs");
 };
 
 // Work item = (head, pair of query tiles).  Same orders as the one-tile kernel:
@@ -122,10 +123,10 @@ __device__ __forceinline__ void pp_issue_pv(uint32_t o_tmem, uint32_t p_tmem, ui
                                             bool first) {
   constexpr uint32_t IDESC_O = C::FP8 ? idesc_e4m3(128, C::D, true) : idesc_bf16(128, C::D, true);
 #pragma unroll
-  for (int kb = 0; kb < C::BN / C::MMA_K; ++kb)
-    umma_ts<C::FP8>(o_tmem, p_tmem + kb * (C::MMA_K * C::ELEM / 4),
-                    vdesc + static_cast<uint64_t>((kb * C::MMA_K * 128) >> 4), IDESC_O,
-                    (first && kb == 0) ? 0u : 1u);
+  for (int kb = 0; kb < C::BN / C::MMA_K; ++kb) {
+    umma_ts<C::FP8>(o_tmem, p_tmem + kb * (C::MMA_K * C::ELEM / 4), vdesc + static_cast<uint64_t>((kb * C::MMA_K * 128) >> 4),
+                    IDESC_O, (first && kb == 0) ? 0u : 1u);
+  }
 }
 
 // ---------------------------------------------------------------- producer (one thread)
@@ -334,9 +335,8 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
     const int n = pp_kv_tiles<C>(p, qt);
     if (n == 0) continue;
     const int q_idx = qt * C::BM + row;
-    constexpr bool kFusedSum = !C::FP8 && ((C::TAU > 0.f && !C::COMP) || C::EXPH);
-    float m = -INFINITY, l = 0.f, lx = 0.f;   // lx: unrounded row sum (fused path)
-    float lc = 0.f;                           // compensated row sum (COMP)
+    float m = -INFINITY, l = 0.f;
+    float lc = 0.f;                           // row sum that normalises O (COMP, RSUM)
     float qsc = 1.f, vmax = 1.f;
     // FP8: the V tile scales' max, one load per lane per 32 tiles and a warp reduction;
     // the per-step K and V scales are fetched a step ahead, so their load latency
@@ -405,101 +405,68 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       }
       const uint64_t c2 = f2_pack(c_j, c_j);
       const uint64_t nm2 = f2_pack(-m_use, -m_use);
+      // Exponentials, their row sum, P packing and the P store per 32-key chunk, so
+      // that packing and the tensor-memory stores overlap the special-function unit.
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-      uint64_t accx[4] = {0ull, 0ull, 0ull, 0ull};   // unrounded sums, fused path
-      // bf16 with TAU > 0 or half-precision exponentials: exponentials, rounding to
-      // bf16 and the row sum of the rounded values in one pass
-      uint32_t pk[C::BN / 2];
-      auto exps_bf16 = [&](auto emu_tag) {
+      uint64_t accr[4] = {0ull, 0ull, 0ull, 0ull};   // RSUM: the rounded probabilities
+      const uint64_t f2fold = f2_pack(fold, fold);
+      auto chunks = [&](auto emu_tag) {
         constexpr int kEmu = decltype(emu_tag)::value;
 #pragma unroll
-        for (int c = 0; c < C::BN; c += 2) {
-          const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c2, nm2);
-          uint64_t p2;
-          if ((c / 2) % 4 < kEmu) {
-            p2 = ex2_poly_pair(x2);
-          } else if constexpr (C::EXPH) {
-            p2 = ex2_f16_pair(x2);
-          } else {
-            float xa, xb;
-            f2_unpack(x2, xa, xb);
-            p2 = f2_pack(ex2(xa), ex2(xb));
-          }
-          float pa, pb;
-          f2_unpack(p2, pa, pb);
-          const uint32_t u = pack_bf16x2(pa, pb);
-          pk[c / 2] = u;
-          acc[(c / 2) % 4] = f2_add(acc[(c / 2) % 4],
-                                    f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
-          accx[(c / 2) % 4] = f2_add(accx[(c / 2) % 4], p2);
-        }
-      };
-      auto exps = [&](auto emu_tag) {
-        constexpr int kEmu = decltype(emu_tag)::value;
+        for (int c0 = 0; c0 < C::BN; c0 += 32) {
+          float pv[32];
 #pragma unroll
-        for (int c = 0; c < C::BN; c += 2) {
-          const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c2, nm2);
-          uint64_t p2;
-          if ((c / 2) % 4 < kEmu) {
-            p2 = ex2_poly_pair(x2);
-          } else {
-            float xa, xb;
-            f2_unpack(x2, xa, xb);
-            p2 = f2_pack(ex2(xa), ex2(xb));
+          for (int i = 0; i < 16; ++i) {
+            const int c = c0 + 2 * i;
+            const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c2, nm2);
+            uint64_t p2;
+            if ((((i + 1) * kEmu) / 16) != ((i * kEmu) / 16)) {
+              p2 = ex2_poly_pair(x2);
+            } else {
+              float xa, xb;
+              f2_unpack(x2, xa, xb);
+              p2 = f2_pack(ex2(xa), ex2(xb));
+            }
+            acc[i % 4] = f2_add(acc[i % 4], p2);
+            if constexpr (C::FP8) p2 = f2_mul(p2, f2fold);
+            f2_unpack(p2, pv[2 * i], pv[2 * i + 1]);
           }
-          acc[(c / 2) % 4] = f2_add(acc[(c / 2) % 4], p2);
-          f2_unpack(p2, s[c], s[c + 1]);
+          if constexpr (C::FP8) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pk[i] = pack_e4m3x4(pv[4 * i], pv[4 * i + 1], pv[4 * i + 2], pv[4 * i + 3]);
+            tmem_st8(lane_base + tm_s + c0 / 4, pk);
+          } else {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              pk[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
+              if constexpr (C::RSUM)
+                accr[i % 4] = f2_add(accr[i % 4], f2_pack(__uint_as_float(pk[i] << 16),
+                                                          __uint_as_float(pk[i] & 0xFFFF0000u)));
+            }
+            tmem_st16(lane_base + tm_s + c0 / 2, pk);
+          }
         }
       };
-      constexpr bool kFused = kFusedSum;
-      if constexpr (kFused) {
-        if (need_mask)
-          exps_bf16(std::integral_constant<int, 0>{});
-        else
-          exps_bf16(std::integral_constant<int, C::EMU>{});
-      } else {
-        if (need_mask)
-          exps(std::integral_constant<int, 0>{});
-        else
-          exps(std::integral_constant<int, C::EMU>{});
-      }
+      if (need_mask)
+        chunks(std::integral_constant<int, 0>{});
+      else
+        chunks(std::integral_constant<int, C::EMU>{});
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
       l = l * alpha + (sa + sb);
       if constexpr (C::COMP) lc = lc * alpha + (sa + sb) + l_comp;
-      if constexpr (kFused) {
-        float xa, xb;
-        f2_unpack(f2_add(f2_add(accx[0], accx[1]), f2_add(accx[2], accx[3])), xa, xb);
-        lx = lx * alpha + (xa + xb);
+      if constexpr (C::RSUM) {
+        float ra, rb;
+        f2_unpack(f2_add(f2_add(accr[0], accr[1]), f2_add(accr[2], accr[3])), ra, rb);
+        lc = lc * alpha + (ra + rb);
       }
-      if constexpr (kFused) {
-#pragma unroll
-        for (int c = 0; c < C::BN / 2; c += 32) {
-          uint32_t r[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = pk[c + i];
-          tmem_st32(lane_base + tm_s + c, r);
-        }
-      } else if constexpr (C::FP8) {
-        uint32_t r[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          r[i] = pack_e4m3x4(s[4 * i] * fold, s[4 * i + 1] * fold, s[4 * i + 2] * fold,
-                             s[4 * i + 3] * fold);
-        tmem_st32(lane_base + tm_s, r);
-      } else {
-#pragma unroll
-        for (int c = 0; c < C::BN; c += 64) {
-          uint32_t r[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = pack_bf16x2(s[c + 2 * i], s[c + 2 * i + 1]);
-          tmem_st32(lane_base + tm_s + c / 2, r);
-        }
-      }
-      // S_t(j) ready => P_t(j-1) V has completed, so O_t may be rescaled now (after
-      // P is stored, when the score row no longer occupies registers).
+      // S_t(j) ready => P_t(j-1) V has completed, so O_t may be rescaled now (after P
+      // is stored, when the score row no longer occupies registers).
       if (j > 0 && __any_sync(0xffffffffu, raise)) {
-        // the whole O row in one TMEM round trip, scaled in packed pairs
+        // the whole O row in one tensor-memory round trip, scaled in packed pairs
         uint32_t r[C::D];
         if constexpr (C::D == 128) {
           tmem_ld128(lane_base + tm_o, r);
@@ -528,7 +495,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       ++gs;
     }
     if (!ok) break;
-    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / (C::COMP ? lc : l);
+    const float inv_l = (C::FP8 ? vmax * (1.f / 256.f) : 1.f) / ((C::COMP || C::RSUM) ? lc : l);
     const bool row_ok = q_idx < p.N;
     if (!(ok = mbar_wait(bar(C::B_ODONE + t), ti & 1, wc, kSiteODone))) break;
     ++ti;
@@ -551,7 +518,7 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
       }
     }
     if (row_ok && p.lse != nullptr)
-      p.lse[static_cast<size_t>(bh) * p.N + q_idx] = (m + __log2f(kFusedSum ? lx : l)) * LN2;
+      p.lse[static_cast<size_t>(bh) * p.N + q_idx] = (m + __log2f(l)) * LN2;
     tc_fence_before();
   }
 }
@@ -572,8 +539,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int warp = threadIdx.x / 32;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NBARS; ++i)
+    for (int i = 0; i < C::NBARS; ++i) {
       mbar_init(bars + 8u * i, (i == C::B_PFULL || i == C::B_PFULL + 1) ? 4u : 1u);  // warps
+    }
     ring.init(C::ITEM_READERS);
     *abort_flag = 0;
     fence_mbar_init();
@@ -591,7 +559,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, p.status, p.timeout_ns};
 
-  if (warp >= 8) {
+  if (warp >= C::SOFTMAX_WARPS) {
     regs_decrease<C::REGS_OTHER>();
     if (warp == C::PRODUCER_WARP && (threadIdx.x & 31) == 0)
       pp_producer<C>(&tq, &tk, &tv, p, sbase, bars, ring, wc);
