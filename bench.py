@@ -619,13 +619,19 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# extra shapes for ncu captures only (not bench lines): the d = 128 backward's passes
+PROFILE_ONLY = {
+    "bwd_d128": workloads.Workload("bwd_d128", 4, 16, 4096, 128, True, backward=True, seed=1006),
+}
+
+
 def run_profile_driver(name, launches):
     """Launch one workload's kernels a few times and exit: the target for ncu captures
     (`ncu --clock-control none -k regex:... -s <skip> -c <n> python bench.py --profile
     <name>`).  Always pass --clock-control none (ncu otherwise locks the GPU clocks),
     and keep a capture beyond gpu__time_duration.sum to one kernel and a few launches."""
     import exact_attention_132_b200 as fa
-    w = workloads.WORKLOADS[name]
+    w = workloads.WORKLOADS[name] if name in workloads.WORKLOADS else PROFILE_ONLY[name]
     dev = torch.device("cuda", 0)
     if w.fp8:
         inp = workloads.make_fp8_inputs(w)
@@ -650,7 +656,7 @@ def run_profile_driver(name, launches):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile", choices=sorted(workloads.WORKLOADS), default=None,
+    ap.add_argument("--profile", choices=sorted(workloads.WORKLOADS) + sorted(PROFILE_ONLY), default=None,
                     help="only launch this workload's kernels (--profile-launches times) for ncu")
     ap.add_argument("--profile-launches", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
