@@ -274,7 +274,7 @@ fa_status launch_fwd_pp(const void* q, const void* k, const void* v, FwdParams p
 #define FA_FWD_D64_EMU 4
 #endif
 #ifndef FA_FWD_F8_EMU
-#define FA_FWD_F8_EMU 4
+#define FA_FWD_F8_EMU 0
 #endif
 #ifndef FA_FWD_D256_EMU
 #define FA_FWD_D256_EMU 0

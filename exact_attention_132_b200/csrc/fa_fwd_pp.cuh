@@ -378,10 +378,14 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
         for (int c = 0; c < C::BN; ++c)
           if (kv0 + c > lim) s[c] = -INFINITY;
       }
-      float c_j = sl2, fold = 1.f;
+      float c_j = sl2, lfold = 0.f, inv_fold = 1.f;
       if constexpr (C::FP8) {
         c_j = sl2 * qsc * ksc;
-        fold = 256.f * vsc / vmax;
+        // P is stored as P~ * fold, fold = 256 * vsc / vmax (reading of the V-scale
+        // folding): the factor enters the exponent, 2^(x + log2 fold), and the row sum
+        // takes it out again once per step
+        lfold = 8.f + __log2f(vsc / vmax);
+        inv_fold = ex2(-lfold);
       }
       // row max: eight independent three-input chains, then a short tree
       float mx[8];
@@ -404,12 +408,11 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
         l_comp = __bfloat162float(__float2bfloat16_rn(pt)) - pt;
       }
       const uint64_t c2 = f2_pack(c_j, c_j);
-      const uint64_t nm2 = f2_pack(-m_use, -m_use);
+      const uint64_t nm2 = f2_pack(lfold - m_use, lfold - m_use);
       // Exponentials, their row sum, P packing and the P store per 32-key chunk, so
       // that packing and the tensor-memory stores overlap the special-function unit.
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       uint64_t accr[4] = {0ull, 0ull, 0ull, 0ull};   // RSUM: the rounded probabilities
-      const uint64_t f2fold = f2_pack(fold, fold);
       auto chunks = [&](auto emu_tag) {
         constexpr int kEmu = decltype(emu_tag)::value;
 #pragma unroll
@@ -428,7 +431,6 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
               p2 = f2_pack(ex2(xa), ex2(xb));
             }
             acc[i % 4] = f2_add(acc[i % 4], p2);
-            if constexpr (C::FP8) p2 = f2_mul(p2, f2fold);
             f2_unpack(p2, pv[2 * i], pv[2 * i + 1]);
           }
           if constexpr (C::FP8) {
@@ -456,6 +458,10 @@ __device__ void pp_softmax(const FwdParams& p, uint32_t bars, uint32_t tmem, int
         chunks(std::integral_constant<int, C::EMU>{});
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
+      if constexpr (C::FP8) {
+        sa *= inv_fold;
+        sb *= inv_fold;
+      }
       l = l * alpha + (sa + sb);
       if constexpr (C::COMP) lc = lc * alpha + (sa + sb) + l_comp;
       if constexpr (C::RSUM) {
