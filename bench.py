@@ -366,9 +366,9 @@ def measure_fp8_peak(dev, gpu):
 
 def run_extras(fa, dev, stream, steps, peak, hbm_peak, gpu):
     """The other workloads of the metric, each with its own clock record and roofline:
-    the small forward (latency), fwd+bwd at the two backward workloads, the headline
-    kernel at N=32768, decoding and the FP8 forward/backward (against a measured FP8
-    matmul peak).  Device-side seeded inputs."""
+    the small forward (latency), fwd+bwd at the two backward workloads and at the
+    headline shape, the headline kernel at N=32768, decoding and the FP8
+    forward/backward (against a measured FP8 matmul peak).  Device-side seeded inputs."""
     out = {}
     src = "measured bf16 dense matmul (burst)"
     gen = torch.Generator(device=dev)
@@ -389,8 +389,11 @@ def run_extras(fa, dev, stream, steps, peak, hbm_peak, gpu):
                         "note": "64 query tiles for 148 SMs: latency-bound, not graded",
                         "roofline": roofline_obj(tf, peak, "TFLOP/s", src), "clocks": clk}
     del q, k, v, o, lse
-    for name in ("fwdbwd_d64", "fwdbwd_d256"):
-        w = workloads.WORKLOADS[name]
+    # the two backward workloads, then the headline shape's own backward (context: d = 128
+    # is the common head dim; its row is not one of the metric's workloads)
+    for name, w in (("fwdbwd_d64", workloads.WORKLOADS["fwdbwd_d64"]),
+                    ("fwdbwd_d256", workloads.WORKLOADS["fwdbwd_d256"]),
+                    ("fwdbwd_d128", PROFILE_ONLY["bwd_d128"])):
         gen.manual_seed(w.seed)
         shp = (w.B, w.H, w.N, w.d)
         q, k, v, do = ((torch.randn(shp, generator=gen, device=dev) * w.std).to(torch.bfloat16)

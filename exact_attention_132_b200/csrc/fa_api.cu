@@ -350,10 +350,19 @@ using FwdF8D256 = FwdCfg<256, 128, 3, 2, true, FA_FWD_F8_EMU>;
 using DkdvD64 = DkdvCfg<64, 64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU>;
 using DkdvD64F =
     DkdvCfg<64, 64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU, true>;
-using DkdvD128 = DkdvCfg<128, 128, 64, 3, 3, 2, 2, FA_BWD_EMU>;
+// d = 128: 128-row query tiles with one S^T and one dP^T buffer (TMEM: 128 + 128 + 2 x 128
+// columns) run ahead of 64-row tiles with two of each: full-width (N = 128) products, half
+// the hand-offs per query row, and S^T(i+1) still overlaps the dS^T(i) work
+#ifndef FA_BWD_D128_EMU
+#define FA_BWD_D128_EMU 1
+#endif
+using DkdvD128 = DkdvCfg<128, 128, 128, 2, 2, 1, 1, FA_BWD_D128_EMU>;
 using DkdvD256 = DkdvCfg<256, 128, 64, 2, 1, 2, 2, FA_BWD_D256_EMU>;
 using DqD64 = DqCfg<64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_EMU>;
-using DqD128 = DqCfg<128, 128, 3, 2, 2, 1, FA_BWD_EMU>;
+#ifndef FA_BWD_DQ128_EMU
+#define FA_BWD_DQ128_EMU FA_BWD_EMU
+#endif
+using DqD128 = DqCfg<128, 128, 3, 2, 2, 1, FA_BWD_DQ128_EMU>;
 using DqD256 = DqCfg<256, 64, 2, 1, 2, 2, FA_BWD_D256_EMU>;
 
 // Launch `kern` as a programmatic dependent of the previous kernel in `stream`: it may

@@ -457,6 +457,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // warps have drained it (after dV(st), below)
     constexpr bool EARLY_S = C::SB == 2 && C::QST >= 2 && !C::FUSEDQ;
     constexpr bool EARLY_DP = EARLY_S && C::DB == 2 && C::OST >= 2;
+    // one S^T buffer: S^T(st+1) goes right behind dV(st), the last reader of P^T(st), so
+    // the tensor core computes it while the compute warps form dS^T(st)
+    constexpr bool S_AFTER_DV = C::SB == 1 && !C::FUSEDQ;
     for (int st = 0; st < nsteps && ok; ++st) {
       const int nx = st + 1;
       // S^T(st+1) into the other buffer (its last reader, dV(st+1-SB), is issued)
@@ -472,6 +475,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       sdesc_sw128(dobuf(st) + hbox * C::BMQ * 128 + kb * 16 * 128, C::BMQ * 128, 1024),
                       ID_G, (st > 0 || kb > 0) ? 1u : 0u);
       tc_commit_elect(bar(C::B_OEMPTY + st % C::OST));     // dP^T(st) and dV(st) read dO(st)
+      if (S_AFTER_DV && nx < nsteps && !(ok = issue_st(nx))) break;
       if constexpr (C::FUSEDQ) {
         if (nx < nsteps) {
           if (st >= 1 &&
@@ -503,7 +507,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       // the next tile's remaining products go after this tile's readers
       if (nx < nsteps) {
-        if (!EARLY_S && !C::FUSEDQ && !(ok = issue_st(nx))) break;
+        if (!EARLY_S && !C::FUSEDQ && !S_AFTER_DV && !(ok = issue_st(nx))) break;
         if (!EARLY_DP && !(ok = issue_dpt(nx))) break;
       }
     }
