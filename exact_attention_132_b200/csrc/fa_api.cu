@@ -362,7 +362,12 @@ using DqD64 = DqCfg<64, 128, FA_BWD_D64_STAGES, FA_BWD_D64_STAGES, 2, 1, FA_BWD_
 #ifndef FA_BWD_DQ128_EMU
 #define FA_BWD_DQ128_EMU FA_BWD_EMU
 #endif
-using DqD128 = DqCfg<128, 128, 3, 2, 2, 1, FA_BWD_DQ128_EMU>;
+// d = 128 dQ pass: one S buffer and two dP buffers (TMEM 128 + 2 x 128 + 128); S(j+1) and
+// dP(j+1) are issued as soon as the compute warps have loaded S(j)
+#ifndef FA_BWD_DQ128_SB
+#define FA_BWD_DQ128_SB 1
+#endif
+using DqD128 = DqCfg<128, 128, 3, 2, FA_BWD_DQ128_SB, 3 - FA_BWD_DQ128_SB, FA_BWD_DQ128_EMU>;
 using DqD256 = DqCfg<256, 64, 2, 1, 2, 2, FA_BWD_D256_EMU>;
 
 // Launch `kern` as a programmatic dependent of the previous kernel in `stream`: it may

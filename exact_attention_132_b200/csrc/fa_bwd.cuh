@@ -722,7 +722,8 @@ struct DqCfg {
                        B_SFULL = 3, B_DPFULL = 3 + SB, B_DS = 3 + SB + DB,
                        B_KFULL = 3 + SB + 2 * DB, B_KEMPTY = B_KFULL + KST,
                        B_VFULL = B_KEMPTY + KST, B_VEMPTY = B_VFULL + VST,
-                       NBARS = B_VEMPTY + VST;
+                       B_SFREE = B_VEMPTY + VST,   // one S buffer: the compute warps loaded S(j)
+                       NBARS = B_SFREE + 1;
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
   static constexpr int TM_S = 0;                 // + b * BN
@@ -761,7 +762,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i)
-      mbar_init(bar(i), (i >= C::B_DS && i < C::B_DS + C::DB) ? 8u : 1u);   // 8 compute warps
+      mbar_init(bar(i), ((i >= C::B_DS && i < C::B_DS + C::DB) || i == C::B_SFREE)
+                            ? 8u : 1u);                     // the 8 compute warps arrive
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -860,10 +862,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       return true;
     };
     // S(j+1) may run ahead of dQ(j): its buffer's last reader, the compute warps'
-    // load of S(j+1-SB), happened before they released dS(j+1-SB).  dP(j+1) has to
-    // follow dQ(j) unless it has a second buffer.
+    // load of S(j+1-SB), happened before they released dS(j+1-SB).  With one S buffer
+    // S(j+1) waits only for that load (the compute warps signal it at once), so it and
+    // the next dP run under the exponentials of tile j.  dP(j+1) has to follow dQ(j)
+    // unless it has a second buffer.
     constexpr bool EARLY_S = C::SB == 2 && C::KST >= 2;
-    constexpr bool EARLY_DP = EARLY_S && C::DB == 2 && C::VST >= 2;
+    constexpr bool S_ON_FREE = C::SB == 1 && C::KST >= 2;
+    constexpr bool EARLY_DP = (EARLY_S || S_ON_FREE) && C::DB == 2 && C::VST >= 2;
     bool ok = mbar_wait_warp(bar(C::B_QDO), 0, wc, kSiteQFull);
     if (ok && nsteps > 0) ok = issue_s(0) && issue_dp(0);
     for (int j = 0; j < nsteps && ok; ++j) {
@@ -871,6 +876,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (EARLY_S && nx < nsteps) {
         // S(nx) overwrites the buffer S(nx - 2) was loaded from: that load preceded
         // dS(nx - 2), which this warp waited for one iteration ago
+        if (!(ok = issue_s(nx))) break;
+        if (EARLY_DP && !(ok = issue_dp(nx))) break;
+      }
+      if (S_ON_FREE && nx < nsteps) {
+        // S(nx) overwrites S(j) once every compute warp has loaded it; dP(nx) goes to
+        // the buffer dQ(j-1), issued one iteration ago, read dS(j-1) from
+        if (!(ok = mbar_wait_warp(bar(C::B_SFREE), j & 1, wc, kSiteSFull))) break;
+        tc_fence_after();
         if (!(ok = issue_s(nx))) break;
         if (EARLY_DP && !(ok = issue_dp(nx))) break;
       }
@@ -885,7 +898,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       (j > 0 || kb > 0) ? 1u : 0u);
       tc_commit_elect(bar(C::B_KEMPTY + j % C::KST));         // S(j) and dQ(j) read K(j)
       if (nx < nsteps) {
-        if (!EARLY_S && !(ok = issue_s(nx))) break;
+        if (!EARLY_S && !S_ON_FREE && !(ok = issue_s(nx))) break;
         if (!EARLY_DP && !(ok = issue_dp(nx))) break;
       }
     }
@@ -918,6 +931,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         } else {
           tmem_ld32(sc, r);
           tmem_ld_wait(r);
+        }
+        if constexpr (C::SB == 1) {            // the MMA warp may now overwrite S(j)
+          tc_fence_before();
+          mbar_arrive_warp(bar(C::B_SFREE));
         }
         exp2_row<C::CH, C::EMU>(r, sl2, lse2, pr);
       }
