@@ -206,15 +206,18 @@ struct DkdvCfg {
                        B_QFULL = 3 + 2 * SB + 2 * DB, B_QEMPTY = B_QFULL + QST,
                        B_OFULL = B_QEMPTY + QST, B_OEMPTY = B_OFULL + OST,
                        B_DQFULL = B_OEMPTY + OST, B_DQFREE = B_DQFULL + 1,
-                       NBARS = B_OEMPTY + OST + (FUSEDQ ? 2 : 0);
+                       B_DQSTG = B_DQFULL + 2,    // fused dQ: the 8 blocks of a step are staged
+                       B_DQSFR = B_DQFULL + 3,    // fused dQ: their reduce-adds have read them
+                       NBARS = B_OEMPTY + OST + (FUSEDQ ? 4 : 0);
   static constexpr int SMEM_MISC = SMEM_BAR + NBARS * 8;
   static constexpr int SMEM_ALLOC = SMEM_MISC + 64 + 1024;
   static constexpr int TM_ST = 0;                        // + b * BMQ
   static constexpr int TM_DPT = SB * BMQ;                // + b * BMQ
   static constexpr int TM_DV = (SB + DB) * BMQ, TM_DK = TM_DV + DH;
   static constexpr int TM_COLS = 512;
-  static constexpr int THREADS = 320;                    // 8 compute warps, producer, MMA
-  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+  // 8 compute warps, producer, MMA; fused dQ: one more warp issues the dQ reduce-adds
+  static constexpr int THREADS = FUSEDQ ? 352 : 320;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, REDUCE_WARP = FUSEDQ ? 10 : -1;
   static_assert((SB + DB) * BMQ + 2 * DH <= TM_COLS, "tensor memory budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(BMQ % 64 == 0 && DH % 64 == 0 && CH % 32 == 0, "box and TMEM chunk sizes");
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBARS; ++i) {
       const bool warps8 = (i >= C::B_P && i < C::B_P + C::SB) || (i >= C::B_DS && i < C::B_DS + C::DB) ||
-                          (C::FUSEDQ && i == C::B_DQFREE);
+                          (C::FUSEDQ && (i == C::B_DQFREE || i == C::B_DQSTG));
       mbar_init(bar(i), warps8 ? 8u : 1u);                  // 8 compute warps arrive
     }
     *abort_flag = 0;
@@ -515,6 +518,28 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     tc_commit_elect(bar(C::B_DRAIN));
     if (!mbar_wait_drain(bar(C::B_DRAIN), 0, wc.timeout_ns) && lane == 0)
       atomicCAS(wc.status, 0u, kStatusTimeout | kSiteDrain);
+  } else if (warp == C::REDUCE_WARP) {
+    // ---------------- fused dQ: per step, the eight staged 32 x 32 blocks of dQ_i go to
+    // the fp32 sums as TMA reduce-adds (issued here, off the compute warps' path); the
+    // compute warps reuse the staging blocks once these have read them
+    bool ok = true;
+    for (int sp = 0; sp < nsteps && ok; ++sp) {
+      if (!(ok = mbar_wait_warp(bar(C::B_DQSTG), sp & 1, wc, kSiteDqDone))) break;
+      if (lane == 0) {
+        const int y0 = q_tile(sp) * C::BMQ;
+        for (int w = 0; w < 8; ++w) {
+          const int y = y0 + (w & 3) * 32;              // rows past N are clipped
+          if (y < p.N)
+            tma_reduce_add_3d(&tdq, sbase + C::SMEM_DQ + w * 4096, (w >> 2) * 32, y, q_head(sp));
+        }
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+      mbar_arrive_warp(bar(C::B_DQSFR));
+    }
+    // the reduce-adds complete before the shared memory goes away and the kernel ends
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   } else {
     // ---------------- compute warps: thread owns key row `row`, query columns of `half`
     const int quad = warp & 3, half = warp >> 2;
@@ -533,22 +558,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tmem_ld_wait(r);
       tc_fence_before();
       mbar_arrive_warp(bar(C::B_DQFREE));          // the columns are free once loaded
-      // staging block: row `lane`, 16-byte chunk c at position c ^ (lane & 7); the
-      // previous reduce-add from it has read it (one step ago)
+      // staging block: row `lane`, 16-byte chunk c at position c ^ (lane & 7), once the
+      // reduce-add of step sp-1 has read it; the reduce warp adds it to the sums
       const uint32_t stg = sbase + C::SMEM_DQ + warp * 4096;
-      if (lane == 0) bulk_wait_read_all();
-      __syncwarp();
+      if (sp > 0 && !mbar_wait(bar(C::B_DQSFR), (sp - 1) & 1, wc, kSiteDqDone)) return false;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         st_shared_v4(stg + lane * 128 + ((c ^ (lane & 7)) << 4), r[4 * c], r[4 * c + 1], r[4 * c + 2],
                      r[4 * c + 3]);
       fence_proxy_async_smem();
-      __syncwarp();
-      const int y = q_tile(sp) * C::BMQ + quad * 32;   // first query row of the block
-      if (lane == 0 && y < p.N) {                        // rows past N are clipped
-        tma_reduce_add_3d(&tdq, stg, half * 32, y, q_head(sp));
-        bulk_commit();
-      }
+      mbar_arrive_warp(bar(C::B_DQSTG));
       return true;
     };
     for (int st = 0; st < nsteps && ok; ++st) {
@@ -676,10 +695,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
         }
       }
-    }
-    // fused dQ: this warp's reduce-adds complete before its shared memory goes away
-    if constexpr (C::FUSEDQ) {
-      if (lane == 0) bulk_wait_all();
     }
   }
 
