@@ -24,14 +24,16 @@
 // At d = 64 (tensor memory has room there) the dK/dV pass also produces dQ:
 //   dQ_i += dS_i K                                      (tensor core, A = dS from smem)
 // accumulated in fp32 in the caller's workspace by TMA reduce-adds (each compute warp
-// stages its 32 x 32 block in shared memory), the sums zeroed by pass 1;
+// stages its 32 x 32 block in shared memory, warp 10 issues the adds), the sums zeroed
+// by pass 1;
 // a fourth kernel, fa_bwd_dq_convert, writes dQ = scale dQ_acc in bf16, and pass 3 is
 // not run (a build choice: the pages give only the recompute).  The fp32 sums' order,
 // and so dQ's last bits, vary from run to run.
 //
 // Roles in kernels 2 and 3: warps 0..7 elementwise work (two warps per TMEM lane
 // quadrant, each on half of the streamed tile's columns), warp 8 TMA producer, warp 9
-// MMA issuer (one elected lane issues; owns tensor memory).
+// MMA issuer (one elected lane issues; owns tensor memory); at d = 64, warp 10 issues
+// the dQ reduce-adds.
 #pragma once
 
 #include "sm100_ptx.cuh"
